@@ -1,0 +1,425 @@
+"""Benchmark of the attention hot path on B200: prefill TFLOP/s and paged-decode KV GB/s.
+
+One step = one pass of the whole path over one batch of synthetic input:
+  1. attn_prefill on the causal MHA GPT-2-small shape (B=8, H=12, S=1024,
+     D=64, bf16; L2 flushed by a 256 MiB write before it), and
+  2. attn_decode_paged on the paged GQA decode batch (64 sequences, Hq=32,
+     Hkv=8, D=128, L ~ U[512, 8192], 16-token pages; 1.1 GB of K/V, larger
+     than L2).
+`value` is the prefill throughput in TFLOP/s (4*D flops per visible
+(query, key) pair); the decode throughput (algorithmic K/V bytes per
+second) is reported beside it with its own roofline.  Each kernel is timed
+with CUDA events on the stream it is launched on.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Under torchrun each rank runs the same per-GPU workload (weak scaling, no
+collective on the data path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from scaled_dot_product_prefill_b200 import inputs, workloads  # noqa: E402
+
+PREFILL = workloads.WORKLOADS["mha_causal_gpt2s"]
+DECODE = workloads.WORKLOADS["paged_decode_gqa"]
+METRIC = "prefill TFLOP/s & paged-decode KV GB/s on 1 B200, % of roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def source_sha(name):
+    p = os.path.join(ROOT, "scaled_dot_product_prefill_b200", "csrc", name)
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload, src):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged since."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    sha = source_sha(src)
+    with open(path) as f:
+        for line in f:
+            parts = line.split("#", 1)[0].split()
+            if len(parts) == 4 and parts[0] == kernel and parts[1] == workload and parts[2] == sha:
+                return int(parts[3])
+    return None
+
+
+# ---------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = []
+        for line in (getattr(self, "out", "") or "").splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), f[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        mx = max(r[1] for r in rows)
+        load = [r for r in rows if r[0] > 0.5 * mx] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in load for i, v in enumerate(r[2]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in load), "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(load)}
+
+
+# ---------------------------------------------------------------- CPU (oracle) legs
+
+
+def cpu_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_prefill_sample(budget_s=8.0):
+    """Float64 oracle on whole (batch, head) slices of the prefill workload until the budget is spent."""
+    from oracle import sdpa
+
+    spec = PREFILL
+    inp = inputs.prefill_inputs(1, 4, 4, spec.Sq, spec.Skv, spec.D, spec.seed)
+    flops = done = 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < budget_s or done == 0:
+        h = done % 4
+        sdpa.attention(inp.q[:, h:h + 1], inp.k[:, h:h + 1], inp.v[:, h:h + 1], spec.scale, spec.causal,
+                       spec.window)
+        flops += workloads.attention_flops(1, 1, spec.Sq, spec.Skv, spec.D, spec.causal, spec.window)
+        done += 1
+    dt = time.perf_counter() - t0
+    return flops / dt / 1e12, f"{done} (batch, head) slices of {spec.name} ({spec.Sq}x{spec.Skv}, D={spec.D})", dt
+
+
+def oracle_decode_sample(budget_s=6.0):
+    from oracle import sdpa
+
+    spec = DECODE
+    p = inputs.paged_inputs(4, spec.Hq, spec.Hkv, spec.D, spec.page_size, spec.seed, len_range=spec.len_range)
+    nbytes = done = 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < budget_s or done == 0:
+        b = done % 4
+        sdpa.decode_paged(p.q[b:b + 1], p.k_pool, p.v_pool, p.page_table[b:b + 1], p.seq_lens[b:b + 1],
+                          spec.page_size, spec.scale, spec.window)
+        nbytes += workloads.kv_bytes(p.seq_lens[b:b + 1].numpy(), spec.Hkv, spec.D)
+        done += 1
+    dt = time.perf_counter() - t0
+    return nbytes / dt / 1e9, f"{done} sequences of {spec.name}", dt
+
+
+# ---------------------------------------------------------------- GPU leg
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    from scaled_dot_product_prefill_b200 import api
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    peaks, peak_kind = load_peaks()
+    spec = PREFILL
+    pi = inputs.prefill_inputs(spec.B, spec.Hq, spec.Hkv, spec.Sq, spec.Skv, spec.D, spec.seed + rank)
+    q, k, v = pi.q.to(dev), pi.k.to(dev), pi.v.to(dev)
+    out = torch.empty_like(q)
+    dspec = DECODE
+    pd = inputs.paged_inputs(dspec.N, dspec.Hq, dspec.Hkv, dspec.D, dspec.page_size, dspec.seed + rank,
+                             len_range=dspec.len_range)
+    dq, kp, vp, pt, sl = (t.to(dev) for t in (pd.q, pd.k_pool, pd.v_pool, pd.page_table, pd.seq_lens))
+    dout = torch.empty_like(dq)
+    msl = pd.max_seq_len
+    ws = torch.empty(api.attn_decode_paged_workspace_size(dspec.N, dspec.Hq, dspec.D, msl, dspec.page_size),
+                     dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    p_flops = workloads.prefill_flops(spec)
+    d_bytes = workloads.decode_bytes(pd.seq_lens.numpy(), dspec.Hq, dspec.Hkv, dspec.D, dspec.page_size)
+    d_kv_bytes = workloads.kv_bytes(pd.seq_lens.numpy(), dspec.Hkv, dspec.D)
+
+    def step(ev=None):
+        flush.zero_()
+        if ev is not None:
+            ev[0].record()
+        api.attn_prefill(q, k, v, causal=spec.causal, window=spec.window, scale=spec.scale, out=out)
+        if ev is not None:
+            ev[1].record()
+            ev[2].record()
+        api.attn_decode_paged(dq, kp, vp, pt, sl, max_seq_len=msl, scale=dspec.scale, window=dspec.window,
+                              workspace=ws, out=dout)
+        if ev is not None:
+            ev[3].record()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    assert api.attn_device_status(clear=True) == 0
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for i in range(args.steps):
+            step(evs[i])
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    assert api.attn_device_status(clear=True) == 0
+    t_pre = [e[0].elapsed_time(e[1]) for e in evs]
+    t_dec = [e[2].elapsed_time(e[3]) for e in evs]
+    pre_ms, dec_ms = float(np.mean(t_pre)), float(np.mean(t_dec))
+    step_ms = pre_ms + dec_ms
+    if dist is not None:
+        tt = torch.tensor([pre_ms, dec_ms, step_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        pre_ms, dec_ms, step_ms = (float(x) for x in tt.tolist())
+
+    # ---- end to end through the public API: pinned host inputs -> device -> kernel -> host result
+    hq, hk, hv = (t.pin_memory() for t in (pi.q, pi.k, pi.v))
+    hout = torch.empty_like(pi.q).pin_memory()
+    e_steps = max(10, args.steps // 10)
+    e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(e_steps)]
+    for i in range(e_steps + 3):
+        flush.zero_()
+        ev = e_ev[i - 3] if i >= 3 else None
+        if ev:
+            ev[0].record()
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        api.attn_prefill(q, k, v, causal=spec.causal, window=spec.window, scale=spec.scale, out=out)
+        hout.copy_(out, non_blocking=True)
+        if ev:
+            ev[1].record()
+    torch.cuda.synchronize()
+    e2e_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in e_ev]))
+    if dist is not None:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = hout.numel() * hout.element_size()
+
+    # ---- the other workloads, one line each (parity cases, reported for context)
+    extra = {}
+    if rank == 0 and not args.no_extra:
+        extra = other_workloads(dev, peaks)
+
+    result = None
+    if rank == 0:
+        tflops = world * p_flops / (pre_ms * 1e-3) / 1e12
+        peak_t = float(peaks["bf16_tflops"])
+        peak_h = float(peaks["hbm_gbs"])
+        ach_t = p_flops / (pre_ms * 1e-3) / 1e12
+        ach_d = d_bytes / (dec_ms * 1e-3) / 1e9
+        traffic = recorded_traffic("prefill_tc_kernel", spec.name, "prefill_sm100.cu")
+        traffic_d = recorded_traffic("decode_split_kernel", dspec.name, "decode_paged.cu")
+        result = {
+            "metric": METRIC,
+            "value": round(tflops, 3),
+            "unit": "TFLOP/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": max(3, args.warmup),
+            "ms_per_step": round(step_ms, 5),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1), bf16)",
+            "config": {
+                "workload": f"{spec.name} + {dspec.name}",
+                "prefill": {"B": spec.B, "Hq": spec.Hq, "Hkv": spec.Hkv, "S": spec.Sq, "D": spec.D,
+                            "causal": spec.causal, "window": spec.window, "flops": p_flops},
+                "decode": {"N": dspec.N, "Hq": dspec.Hq, "Hkv": dspec.Hkv, "D": dspec.D,
+                           "page_size": dspec.page_size, "len_range": list(dspec.len_range),
+                           "sum_len": int(pd.seq_lens.sum()), "kv_bytes": d_kv_bytes, "bytes": d_bytes},
+                "l2": "prefill: 256 MiB write before each call; decode: 1.1 GB K/V > 126 MB L2",
+                "parallelism": f"replicas x{world}",
+            },
+            "roofline": {"bound": "tensor", "achieved": round(ach_t, 2), "peak": peak_t, "unit": "TFLOP/s",
+                         "frac": round(ach_t / peak_t, 4), "traffic": traffic,
+                         "kernel": "prefill_tc_kernel<64>", "peak_kind": f"bf16 burst, {peak_kind}"},
+            "roofline_decode": {"bound": "hbm", "achieved": round(ach_d, 1), "peak": peak_h, "unit": "GB/s",
+                                "frac": round(ach_d / peak_h, 4), "traffic": traffic_d,
+                                "kernel": "decode_split_kernel<128,4> + decode_combine_kernel<128>",
+                                "peak_kind": f"HBM copy, {peak_kind}"},
+            "decode": {"value": round(world * d_bytes / (dec_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                       "ms": round(dec_ms, 5)},
+            "prefill_ms": round(pre_ms, 5),
+            "e2e": {"value": round(world * p_flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms": round(e2e_ms, 5),
+                    "path": "pinned host q/k/v -> device, attn_prefill, out -> pinned host"},
+            "gpu_launches": 3 * args.steps,
+            "clocks": clk.summary(),
+            "workloads": extra,
+        }
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+def time_call(fn, reps, flush=None):
+    import torch
+
+    for _ in range(3):
+        fn()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
+    for e in ev:
+        if flush is not None:
+            flush.zero_()
+        e[0].record()
+        fn()
+        e[1].record()
+    torch.cuda.synchronize()
+    return float(np.median([a.elapsed_time(b) for a, b in ev]))
+
+
+def other_workloads(dev, peaks):
+    import torch
+
+    from scaled_dot_product_prefill_b200 import api
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    res = {}
+    for name, spec in workloads.WORKLOADS.items():
+        if not isinstance(spec, workloads.PrefillSpec):
+            continue
+        pi = inputs.prefill_inputs(spec.B, spec.Hq, spec.Hkv, spec.Sq, spec.Skv, spec.D, spec.seed, spec.dtype)
+        q, k, v = pi.q.to(dev), pi.k.to(dev), pi.v.to(dev)
+        out = torch.empty_like(q)
+        fn = api.attn_prefill if spec.dtype == "bf16" else api.attn_prefill_f32
+        ms = time_call(lambda: fn(q, k, v, causal=spec.causal, window=spec.window, scale=spec.scale, out=out),
+                       20, flush)
+        fl = workloads.prefill_flops(spec)
+        ach = fl / (ms * 1e-3) / 1e12
+        entry = {"ms": round(ms, 5), "TFLOP/s": round(ach, 2)}
+        if spec.dtype == "bf16":
+            entry["frac_of_bf16_peak"] = round(ach / float(peaks["bf16_tflops"]), 4)
+        res[name] = entry
+        del q, k, v, out
+    torch.cuda.empty_cache()
+    return res
+
+
+def reference_line(args, rank, world):
+    """The float64 oracle on the host cores, on a bounded sample of the same workload."""
+    if rank != 0:
+        return None
+    threads = cpu_threads()
+    per_step = []
+    for _ in range(max(1, args.steps) + max(0, min(args.warmup, 1))):
+        v, sample, dt = oracle_prefill_sample(budget_s=min(10.0, 60.0 / max(1, args.steps)))
+        per_step.append(v)
+    v = float(np.mean(per_step[-max(1, args.steps):]))
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1), bf16 values upcast)",
+        "config": {"workload": f"{PREFILL.name} (oracle sample)", "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(v, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", args.gpus if args.gpus == 1 else 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    threads = cpu_threads()
+    os.environ.setdefault("OMP_NUM_THREADS", str(threads))
+
+    if args.impl == "reference":
+        line = reference_line(args, rank, world)
+        if line is not None:
+            print(json.dumps(line))
+        return
+
+    result = run_ours(args, rank, world, local_rank)
+    if rank == 0:
+        if not args.no_cpu_baseline and world == 1:
+            v, sample, dt = oracle_prefill_sample()
+            vd, sample_d, dtd = oracle_decode_sample()
+            result["cpu_baseline"] = {"value": round(v, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                                      "sample": sample, "seconds": round(dt, 2),
+                                      "decode": {"value": round(vd, 4), "unit": "GB/s", "sample": sample_d,
+                                                 "seconds": round(dtd, 2)}}
+        print(json.dumps(result))
+
+
+if __name__ == "__main__":
+    main()

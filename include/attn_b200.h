@@ -1,0 +1,181 @@
+/*
+ * attn_b200.h -- C ABI of libattn_b200.so: exact scaled-dot-product attention
+ * on NVIDIA B200 (sm_100a).
+ *
+ *     O = softmax(Q K^T * scale + mask) V
+ *
+ * The operation is the one every source page turns on: "Attention mechanism
+ * explained: from Self-Attention to Multi-Query Attention" (guijiagi.com),
+ * section 2.1 (the formula) and 2.2 (masked_fill with -inf before softmax);
+ * "Taking LLMs apart (2): attention by hand" (blog.kerro.cn), sections
+ * "full implementation" (mask True = visible, masked logits -inf) and
+ * "FlashAttention" (tiled evaluation with an online softmax gives the exact
+ * same result).  Two forms are provided:
+ *
+ *   attn_prefill / attn_prefill_f32   tiled, FlashAttention-style prefill
+ *                                     ("Attention From Scratch" project
+ *                                     README, section "Flash Attention";
+ *                                     the Attention-mechanism explainer,
+ *                                     section 7) with causal and
+ *                                     sliding-window masks ("LLM core
+ *                                     technology", section "Sliding Window
+ *                                     Attention") and MHA/GQA/MQA head sharing
+ *                                     (explainer, sections 4-5).
+ *   attn_decode_paged                 one query token per sequence against a
+ *                                     paged KV cache ("Attention From
+ *                                     Scratch" README, sections "KV Cache"
+ *                                     and "Paged KV Cache"; "LLM core
+ *                                     technology", section "PagedAttention").
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Pointers named q, k, v, out, k_pool, v_pool, page_table, seq_lens and
+ *   workspace are DEVICE pointers of the current CUDA device, 16-byte
+ *   aligned, owned by the caller.  The library never allocates or frees
+ *   device memory and keeps no state between calls (re-entrant).
+ * - bf16 means IEEE bfloat16 stored in 16 bits; inputs are read as bf16,
+ *   all arithmetic accumulates in fp32, outputs are rounded to bf16 with
+ *   round-to-nearest-even.
+ * - Calls are asynchronous on `stream` (NULL = legacy default stream).  The
+ *   return value covers argument validation and the launch itself; a fault
+ *   inside a kernel surfaces at the caller's next synchronisation.
+ * - A zero-sized problem (B, N, Sq or Hq equal to 0) returns ATTN_OK and
+ *   launches nothing.
+ * - Masks.  With Sq query rows and Skv keys, off = Skv - Sq (bottom-right
+ *   alignment).  Non-causal: every key is visible.  Causal: key j is visible
+ *   to row i iff j <= i + off.  window W > 0 (causal only) additionally
+ *   requires j > i + off - W: the query's own position and the W-1 before
+ *   it.  A row with no visible key produces 0.
+ * - GQA: query head h reads kv head h / (Hq / Hkv) (contiguous groups, the
+ *   repeat_interleave order of the explainer's section 5.2); Hq must be a
+ *   multiple of Hkv.  Hkv == Hq is MHA, Hkv == 1 is MQA.
+ * - Device-side waits are bounded.  A kernel that gives up waiting, or that
+ *   meets a page-table entry outside the pool, records it in a device error
+ *   word and skips the affected work instead of faulting or hanging;
+ *   attn_device_status() reads (and optionally clears) that word.
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream; declared here so that callers
+ * need no CUDA header. */
+typedef struct CUstream_st* attn_stream_t;
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1,   /* null pointer, negative size, Hq % Hkv != 0, misaligned pointer */
+  ATTN_ERR_UNSUPPORTED = 2,   /* valid but not implemented: head dim, page size, group size,
+                                 window without causal */
+  ATTN_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed (launch, descriptor, device query) */
+  ATTN_ERR_TIMEOUT = 4,       /* a device-side wait gave up (reported by attn_device_status) */
+  ATTN_ERR_BAD_PAGE = 5,      /* a page-table entry was outside [0, num_pages), or a sequence was
+                                 longer than max_pages * page_size or max_seq_len
+                                 (reported by attn_device_status) */
+  ATTN_ERR_WORKSPACE = 6      /* workspace missing or smaller than attn_decode_paged_workspace_size */
+} attn_status_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* attn_status_string(attn_status_t status);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int attn_version(void);
+
+/*
+ * attn_prefill -- bf16 tiled prefill on the sm_100a tensor cores.
+ *
+ * q   : [B, Hq,  Sq,  D] bf16, contiguous (row-major, D innermost)
+ * k, v: [B, Hkv, Skv, D] bf16, contiguous
+ * out : [B, Hq,  Sq,  D] bf16, contiguous; must not alias q, k or v
+ * D   : 64 or 128 (otherwise ATTN_ERR_UNSUPPORTED)
+ * scale : multiplier of q.k (1/sqrt(D) in the pages; passed explicitly)
+ * causal: 0 or 1;  window: 0 = none, > 0 = sliding window (needs causal=1)
+ *
+ * Q.K^T and P.V run as tcgen05 MMAs (bf16 x bf16 -> fp32 in tensor memory)
+ * on tiles staged by TMA; the softmax is the online form (running row max
+ * and sum, accumulator rescaled when the max grows) and P is rounded to
+ * bf16 before P.V.  Key tiles that the mask hides entirely are skipped.
+ * Errors: ATTN_ERR_INVALID_ARG for null/misaligned pointers or bad sizes,
+ * ATTN_ERR_UNSUPPORTED for D not in {64,128} or window>0 without causal,
+ * ATTN_ERR_CUDA if the tensor-map encoder or the launch fails.
+ */
+attn_status_t attn_prefill(const void* q, const void* k, const void* v, void* out,
+                           int B, int Hq, int Hkv, int Sq, int Skv, int D,
+                           float scale, int causal, int window, attn_stream_t stream);
+
+/*
+ * attn_prefill_f32 -- the same operation with fp32 inputs and output, fp32
+ * arithmetic throughout (FFMA on the CUDA cores; no TF32), for results
+ * that must agree with a float64 evaluation to about 1e-5.
+ *
+ * q : [B, Hq, Sq, D] float; k, v: [B, Hkv, Skv, D] float; out: [B, Hq, Sq, D] float.
+ * D : 64 or 128.  Other arguments and errors as attn_prefill.
+ */
+attn_status_t attn_prefill_f32(const float* q, const float* k, const float* v, float* out,
+                               int B, int Hq, int Hkv, int Sq, int Skv, int D,
+                               float scale, int causal, int window, attn_stream_t stream);
+
+/*
+ * attn_decode_paged -- one decode step for N sequences over a paged KV cache.
+ *
+ * q          : [N, Hq, D] bf16, the new token's query of every sequence
+ * k_pool     : [num_pages, Hkv, page_size, D] bf16, shared page pool
+ * v_pool     : [num_pages, Hkv, page_size, D] bf16
+ * page_table : [N, max_pages] int32; entry p of row b is the physical page
+ *              holding tokens [p*page_size, (p+1)*page_size) of sequence b.
+ *              Entries past a sequence's last page are never read.
+ * seq_lens   : [N] int32 (device), tokens in each cache INCLUDING the new
+ *              token (its k/v are already appended); 0 gives a zero output.
+ * page_size  : tokens per page, a multiple of 16 in [16, 256]
+ * max_seq_len: host-side upper bound of seq_lens, used only to size the
+ *              split-KV grid; longer sequences are reported as
+ *              ATTN_ERR_BAD_PAGE by attn_device_status and truncated.
+ * window     : 0 = attend to all seq_lens[b] keys; W > 0 = the last W keys.
+ * workspace  : device scratch of at least
+ *              attn_decode_paged_workspace_size(N, Hq, D, max_seq_len, page_size)
+ *              bytes, 16-byte aligned; the call uses it for the per-split
+ *              partial outputs and log-sum-exps; contents are not needed
+ *              between calls.  Two calls in flight at once need two
+ *              workspaces.
+ * out        : [N, Hq, D] bf16
+ * D = 128 or 64; Hq / Hkv in {1, 2, 4, 8, 16}.
+ *
+ * Two kernels run on `stream`: a split-KV pass (one CTA per sequence, kv
+ * head and span of keys; the query heads of a GQA group share every K/V
+ * page read; pages are fetched whole by bulk asynchronous copies through
+ * the page table) and a combine pass that merges the splits by their
+ * log-sum-exp.  Errors: ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED,
+ * ATTN_ERR_WORKSPACE, ATTN_ERR_CUDA.
+ */
+attn_status_t attn_decode_paged(const void* q, const void* k_pool, const void* v_pool,
+                                const int32_t* page_table, const int32_t* seq_lens,
+                                int page_size, int N, int Hq, int Hkv, int D,
+                                int num_pages, int max_pages, int max_seq_len,
+                                float scale, int window,
+                                void* workspace, size_t workspace_bytes,
+                                void* out, attn_stream_t stream);
+
+/* Bytes of workspace attn_decode_paged needs for these sizes (0 if any size
+ * is invalid).  Pure host arithmetic, no CUDA call. */
+size_t attn_decode_paged_workspace_size(int N, int Hq, int D, int max_seq_len, int page_size);
+
+/*
+ * attn_device_status -- read the device error word of the current device
+ * (synchronises the device).  Returns ATTN_OK if no kernel has recorded an
+ * error since the last clear, ATTN_ERR_TIMEOUT if a bounded wait gave up,
+ * ATTN_ERR_BAD_PAGE if a page-table entry or sequence length was out of
+ * range, ATTN_ERR_CUDA if the read itself failed.  clear != 0 resets the word.
+ */
+attn_status_t attn_device_status(int clear);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H */

@@ -1,0 +1,146 @@
+// attn_api.cu -- the extern "C" entry points declared in include/attn_b200.h:
+// argument validation, the per-device error word, and dispatch to the
+// kernel launchers.  No device memory is allocated here or anywhere in the
+// library.
+#include <cmath>
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <mutex>
+
+#include "attn_b200.h"
+#include "common.cuh"
+
+namespace attn {
+
+// One error word per device that has loaded the library.
+__device__ unsigned int g_error_word = 0;
+
+unsigned int* device_error_word() {
+  constexpr int kMaxDevices = 64;
+  static unsigned int* addr[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<unsigned int*>(p);
+  }
+  return addr[dev];
+}
+
+}  // namespace attn
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+attn_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA; }
+
+attn_status_t check_prefill(const void* q, const void* k, const void* v, const void* out, int B, int Hq, int Hkv,
+                            int Sq, int Skv, int D, float scale, int causal, int window) {
+  if (B < 0 || Hq < 0 || Hkv < 0 || Sq < 0 || Skv < 0 || D <= 0 || window < 0) return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (B == 0 || Hq == 0 || Sq == 0) return ATTN_OK;  // nothing to do (checked again by the caller)
+  if (Hkv == 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (window > 0 && !causal) return ATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * Hq > 65535LL * 32768LL) return ATTN_ERR_UNSUPPORTED;
+  return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* attn_status_string(attn_status_t s) {
+  switch (s) {
+    case ATTN_OK: return "ATTN_OK";
+    case ATTN_ERR_INVALID_ARG: return "ATTN_ERR_INVALID_ARG";
+    case ATTN_ERR_UNSUPPORTED: return "ATTN_ERR_UNSUPPORTED";
+    case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA";
+    case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT";
+    case ATTN_ERR_BAD_PAGE: return "ATTN_ERR_BAD_PAGE";
+    case ATTN_ERR_WORKSPACE: return "ATTN_ERR_WORKSPACE";
+  }
+  return "ATTN_ERR_UNKNOWN";
+}
+
+int attn_version(void) { return 100; }
+
+attn_status_t attn_prefill(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv, int Sq,
+                           int Skv, int D, float scale, int causal, int window, attn_stream_t stream) {
+  const attn_status_t st = check_prefill(q, k, v, out, B, Hq, Hkv, Sq, Skv, D, scale, causal, window);
+  if (st != ATTN_OK || B == 0 || Hq == 0 || Sq == 0) return st;
+  if (Skv == 0)  // no key at all: every row is empty and its output is 0
+    return from_cuda(cudaMemsetAsync(out, 0, static_cast<size_t>(B) * Hq * Sq * D * 2,
+                                     reinterpret_cast<cudaStream_t>(stream)));
+  return from_cuda(attn::launch_prefill_tc(q, k, v, out, B, Hq, Hkv, Sq, Skv, D, scale, causal, window,
+                                           attn::device_error_word(), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+attn_status_t attn_prefill_f32(const float* q, const float* k, const float* v, float* out, int B, int Hq, int Hkv,
+                               int Sq, int Skv, int D, float scale, int causal, int window, attn_stream_t stream) {
+  const attn_status_t st = check_prefill(q, k, v, out, B, Hq, Hkv, Sq, Skv, D, scale, causal, window);
+  if (st != ATTN_OK || B == 0 || Hq == 0 || Sq == 0) return st;
+  if (static_cast<long long>(B) * Hq > 65535) return ATTN_ERR_UNSUPPORTED;
+  if (Skv == 0)
+    return from_cuda(cudaMemsetAsync(out, 0, static_cast<size_t>(B) * Hq * Sq * D * sizeof(float),
+                                     reinterpret_cast<cudaStream_t>(stream)));
+  return from_cuda(attn::launch_prefill_f32(q, k, v, out, B, Hq, Hkv, Sq, Skv, D, scale, causal, window,
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t attn_decode_paged_workspace_size(int N, int Hq, int D, int max_seq_len, int page_size) {
+  if (N < 0 || Hq < 0 || D <= 0 || max_seq_len < 0 || page_size <= 0) return 0;
+  return attn::decode_workspace_bytes(N, Hq, D, max_seq_len, page_size);
+}
+
+attn_status_t attn_decode_paged(const void* q, const void* k_pool, const void* v_pool, const int32_t* page_table,
+                                const int32_t* seq_lens, int page_size, int N, int Hq, int Hkv, int D,
+                                int num_pages, int max_pages, int max_seq_len, float scale, int window,
+                                void* workspace, size_t workspace_bytes, void* out, attn_stream_t stream) {
+  if (N < 0 || Hq < 0 || Hkv < 0 || D <= 0 || num_pages < 0 || max_pages < 0 || max_seq_len < 0 || window < 0 ||
+      page_size <= 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (N == 0 || Hq == 0) return ATTN_OK;
+  if (Hkv == 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (q == nullptr || out == nullptr || seq_lens == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (max_seq_len > 0 && (k_pool == nullptr || v_pool == nullptr || page_table == nullptr || max_pages == 0))
+    return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(page_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+    return ATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return ATTN_ERR_UNSUPPORTED;
+  if (page_size % 16 != 0 || page_size > 256) return ATTN_ERR_UNSUPPORTED;
+  if (N > 65535 || Hkv > 65535) return ATTN_ERR_UNSUPPORTED;
+  const size_t need = attn::decode_workspace_bytes(N, Hq, D, max_seq_len, page_size);
+  if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)) return ATTN_ERR_WORKSPACE;
+  return from_cuda(attn::launch_decode_paged(q, k_pool, v_pool, page_table, seq_lens, page_size, N, Hq, Hkv, D,
+                                             num_pages, max_pages, max_seq_len, scale, window, workspace, out,
+                                             attn::device_error_word(), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+attn_status_t attn_device_status(int clear) {
+  unsigned int* addr = attn::device_error_word();
+  if (addr == nullptr) return ATTN_ERR_CUDA;
+  unsigned int word = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaMemcpy(&word, addr, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (clear) {
+    const unsigned int zero = 0;
+    if (cudaMemcpy(addr, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  if (word & ATTN_ERRBIT_TIMEOUT) return ATTN_ERR_TIMEOUT;
+  if (word & ATTN_ERRBIT_BADPAGE) return ATTN_ERR_BAD_PAGE;
+  return ATTN_OK;
+}
+
+}  // extern "C"

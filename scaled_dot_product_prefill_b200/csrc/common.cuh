@@ -1,0 +1,46 @@
+// common.cuh -- definitions shared by the kernels and the host API.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+// Upper bound of any single device-side wait (1 s).  No legitimate wait in
+// these kernels lasts more than a few microseconds.
+#ifndef ATTN_WAIT_NS
+#define ATTN_WAIT_NS 1000000000ull
+#endif
+
+#define ATTN_ERRBIT_TIMEOUT 1u   // a bounded wait gave up
+#define ATTN_ERRBIT_BADPAGE 2u   // a page-table entry outside the pool, or seq_len too long
+
+namespace attn {
+
+// Kernels receive a pointer to the per-device error word kept by the API
+// translation unit and OR error bits into it.
+__device__ __forceinline__ void record_error(unsigned int* err, unsigned int bit) {
+  if (err != nullptr) atomicOr(err, bit);
+}
+
+// Device address of this device's error word (looked up once per device).
+unsigned int* device_error_word();
+
+// Host-side launchers (defined next to their kernels).
+cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv,
+                              int Sq, int Skv, int D, float scale, int causal, int window,
+                              unsigned int* err, cudaStream_t stream);
+cudaError_t launch_prefill_f32(const float* q, const float* k, const float* v, float* out, int B, int Hq,
+                               int Hkv, int Sq, int Skv, int D, float scale, int causal, int window,
+                               cudaStream_t stream);
+
+struct DecodeGeometry {
+  int split_tokens;   // keys per split (multiple of 64)
+  int max_splits;     // splits per sequence for max_seq_len
+};
+DecodeGeometry decode_geometry(int N, int Hq, int D, int max_seq_len, int page_size);
+size_t decode_workspace_bytes(int N, int Hq, int D, int max_seq_len, int page_size);
+cudaError_t launch_decode_paged(const void* q, const void* k_pool, const void* v_pool, const int32_t* page_table,
+                                const int32_t* seq_lens, int page_size, int N, int Hq, int Hkv, int D,
+                                int num_pages, int max_pages, int max_seq_len, float scale, int window,
+                                void* workspace, void* out, unsigned int* err, cudaStream_t stream);
+
+}  // namespace attn

@@ -1,0 +1,486 @@
+// decode_paged.cu -- one decode step over a paged KV cache (split-KV + combine).
+//
+// What is computed: for every sequence b and query head h (kv head
+// g = h / G, G = Hq / Hkv), o = softmax(K_b q * scale) V_b over the keys
+// [lo, L) of the sequence's cache, L = seq_lens[b], lo = max(0, L - window)
+// (lo = 0 without a window).  Token t lives in physical page
+// page_table[b][t / page_size] at slot t % page_size ("Attention From
+// Scratch" README, section "Paged KV Cache": fixed-size pages, per-sequence
+// page tables, one shared pool; "LLM core technology", section
+// "PagedAttention").  The cache already holds the new token, so no causal
+// mask is needed ("Taking LLMs apart (2)", section "KV cache").
+//
+// How: decode is bound by HBM bandwidth (every K/V byte is read once per kv
+// head and used for 2*G flops), so the design goal is bytes in flight and
+// no wasted reads; tensor cores play no part.
+//
+// * decode_split_kernel: grid (split, kv head, sequence).  Each CTA owns a
+//   span of `split_tokens` keys; its four warps take interleaved 16-token
+//   chunks.  A chunk of one kv head is 16 * D contiguous bf16 (4 KB at
+//   D = 128) inside one page, so each warp fetches K and V chunks with two
+//   bulk asynchronous copies into its own shared-memory ring and never
+//   stalls on individual loads.  Page-table entries for the warp's chunks
+//   are read once, one per lane, up front.  All G query heads of the group
+//   are evaluated against each K/V element while it is in registers.
+//   The online softmax keeps a reference maximum per head and only moves it
+//   (rescaling the running sum and accumulator) when a score exceeds it by
+//   more than 2^8 in probability, which leaves the result exact.  Each
+//   split writes its normalised partial output and base-2 log-sum-exp.
+// * decode_combine_kernel: one warp per (sequence, head) merges the splits,
+//   weighting each by 2^(lse_s - max lse) ("Attention From Scratch"
+//   README, section "Flash Attention": the pair (output, lse)).
+#include <cmath>
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "sm100_ptx.cuh"
+
+namespace attn {
+namespace {
+
+constexpr int kWarps = 4;       // warps per split CTA
+constexpr int kChunk = 16;      // tokens per chunk (one bulk copy per K and per V)
+constexpr float kTau = 8.0f;    // lazy-rescale threshold, log2 units
+
+struct DecodeParams {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k_pool;
+  const __nv_bfloat16* v_pool;
+  const int32_t* page_table;
+  const int32_t* seq_lens;
+  float* ws_o;        // [N, Hq, max_splits, D]
+  float* ws_lse;      // [N, Hq, max_splits]
+  __nv_bfloat16* out; // [N, Hq, D]
+  unsigned int* err;
+  int page_size, Hq, Hkv, num_pages, max_pages, max_seq_len;
+  int split_tokens, max_splits, window;
+  float scale_log2;
+};
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+// Sum NV per-lane values over groups of R lanes (lane bits below R) and
+// leave each lane with max(1, NV / R) fully reduced values; `base` returns
+// the original index of the lane's first value.
+template <int NV, int R>
+__device__ __forceinline__ void reduce_scatter(float (&v)[NV], int lane, int& base) {
+  base = 0;
+  int n = NV;
+#pragma unroll
+  for (int m = R / 2; m >= 1; m >>= 1) {
+    if (n > 1) {
+      const int half = n / 2;
+      const bool upper = (lane & m) != 0;
+#pragma unroll
+      for (int j = 0; j < NV / 2; ++j) {
+        if (j < half) {
+          const float send = upper ? v[j] : v[half + j];
+          const float keep = upper ? v[half + j] : v[j];
+          v[j] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+        }
+      }
+      base += upper ? half : 0;
+      n = half;
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], m);
+    }
+  }
+}
+
+template <int D>
+struct Geo {
+  static constexpr int R = D / 8;                 // lanes per token row (16 B each)
+  static constexpr int TPL = 32 / R;              // tokens per warp-wide 16 B load
+  static constexpr int NL = kChunk / TPL;         // loads per chunk per lane
+  static constexpr int CHUNK_BYTES = kChunk * D * 2;
+  static constexpr int STAGES = (D == 128) ? 3 : 4;
+};
+
+template <int D, int G>
+struct SplitSmem {
+  alignas(1024) uint8_t ring[kWarps][Geo<D>::STAGES][2][Geo<D>::CHUNK_BYTES];  // K then V
+  alignas(16) float pbuf[kWarps][kChunk * G];     // p of the current chunk, [token][head]
+  float wm[kWarps][G];                            // per-warp reference max (log2 units)
+  float wl[kWarps][G];                            // per-warp running sum
+  uint64_t full[kWarps][Geo<D>::STAGES];
+  int stage_ok[kWarps][Geo<D>::STAGES];
+};
+
+template <int D, int G>
+__global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(const DecodeParams p) {
+  using Gm = Geo<D>;
+  constexpr int R = Gm::R, TPL = Gm::TPL, NL = Gm::NL, STAGES = Gm::STAGES;
+  constexpr int NV = NL * G;                       // partial dot products per lane per chunk
+  constexpr int NF = (NV / R) > 0 ? (NV / R) : 1;  // scores held per lane after reduction
+  constexpr int DUP = (NV >= R) ? 1 : R / NV;       // lanes sharing one score when NV < R
+  extern __shared__ uint8_t smem_raw[];
+  SplitSmem<D, G>& sm = *reinterpret_cast<SplitSmem<D, G>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+  const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  int L = p.seq_lens[b];
+  if (L > p.max_seq_len || L > p.max_pages * p.page_size) {
+    if (threadIdx.x == 0 && s == 0) record_error(p.err, ATTN_ERRBIT_BADPAGE);
+    L = min(L, min(p.max_seq_len, p.max_pages * p.page_size));
+  }
+  if (L <= 0) return;
+  const int lo = (p.window > 0) ? max(0, L - p.window) : 0;
+  if (s < lo / p.split_tokens || s > (L - 1) / p.split_tokens) return;  // split holds no visible key
+
+  const int t_begin = max(s * p.split_tokens, lo);
+  const int t_end = min((s + 1) * p.split_tokens, L);
+  const int c_begin = t_begin / kChunk;
+  const int c_end = (t_end + kChunk - 1) / kChunk;
+  // chunks of this warp: c_begin + warp + kWarps * i
+  const int n_my = (c_end - c_begin - warp + kWarps - 1) / kWarps;  // may be <= 0
+
+  if (threadIdx.x < kWarps * STAGES) {
+    mbar_init(&sm.full[threadIdx.x / STAGES][threadIdx.x % STAGES], 1);
+  }
+  fence_mbar_init();
+  __syncthreads();
+
+  const size_t head_stride = static_cast<size_t>(p.page_size) * D;  // elements per (page, head)
+  // lane i holds the physical page of the warp's i-th chunk
+  int my_page = -1;
+  if (lane < n_my) {
+    const int t0 = (c_begin + warp + kWarps * lane) * kChunk;
+    my_page = p.page_table[static_cast<size_t>(b) * p.max_pages + t0 / p.page_size];
+  }
+
+  auto issue = [&](int i) {  // whole warp calls; lane 0 issues chunk i into stage i % STAGES
+    const int phys = __shfl_sync(0xffffffffu, my_page, i);
+    if (lane == 0) {
+      const int st = i % STAGES;
+      uint64_t* bar = &sm.full[warp][st];
+      if (phys < 0 || phys >= p.num_pages) {
+        record_error(p.err, ATTN_ERRBIT_BADPAGE);
+        sm.stage_ok[warp][st] = 0;
+        mbar_arrive(bar);
+      } else {
+        sm.stage_ok[warp][st] = 1;
+        const int t0 = (c_begin + warp + kWarps * i) * kChunk;
+        const size_t off = (static_cast<size_t>(phys) * p.Hkv + g) * head_stride +
+                           static_cast<size_t>(t0 % p.page_size) * D;
+        mbar_arrive_expect_tx(bar, 2 * Gm::CHUNK_BYTES);
+        bulk_load(sm.ring[warp][st][0], p.k_pool + off, Gm::CHUNK_BYTES, bar);
+        bulk_load(sm.ring[warp][st][1], p.v_pool + off, Gm::CHUNK_BYTES, bar);
+      }
+    }
+  };
+
+  const int n_pro = min(n_my, STAGES);
+  for (int i = 0; i < n_pro; ++i) issue(i);
+
+  // query of the G heads of this group, my 8 columns, pre-scaled to log2 units
+  const int d0 = (lane % R) * 8;
+  float qf[G][8];
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh) {
+    const uint4 u = *reinterpret_cast<const uint4*>(
+        p.q + (static_cast<size_t>(b) * p.Hq + g * G + hh) * D + d0);
+    bf16x8_to_f32(u, qf[hh]);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) qf[hh][e] *= p.scale_log2;
+  }
+
+  float m_ref[G], l_part[G], acc[G][8];
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh) {
+    m_ref[hh] = -INFINITY;
+    l_part[hh] = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[hh][e] = 0.f;
+  }
+
+  bool ok_all = true;
+  for (int i = 0; i < n_my; ++i) {
+    const int st = i % STAGES;
+    if (!mbar_wait(&sm.full[warp][st], (i / STAGES) & 1, nullptr, p.err)) {
+      // give the copies still in flight a bounded chance to land before the ring is reused
+      for (int k = i + 1; k < min(n_my, i + STAGES); ++k)
+        mbar_wait(&sm.full[warp][k % STAGES], (k / STAGES) & 1, nullptr, p.err);
+      ok_all = false;
+      break;
+    }
+    const int chunk_t0 = (c_begin + warp + kWarps * i) * kChunk;
+    const bool stage_ok = sm.stage_ok[warp][st] != 0;
+    const bool full = stage_ok && chunk_t0 >= lo && chunk_t0 + kChunk <= L;
+    const uint4* sk = reinterpret_cast<const uint4*>(sm.ring[warp][st][0]);
+    const uint4* sv = reinterpret_cast<const uint4*>(sm.ring[warp][st][1]);
+
+    // ---- scores: partial dot products over my 8 columns, then reduce over the row's R lanes
+    float part[NV];
+#pragma unroll
+    for (int l = 0; l < NL; ++l) {
+      float kf[8];
+      bf16x8_to_f32(sk[l * 32 + lane], kf);
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) {
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) a = fmaf(qf[hh][e], kf[e], a);
+        part[l * G + hh] = a;
+      }
+    }
+    int base;
+    reduce_scatter<NV, R>(part, lane, base);
+
+    // my NF scores: index idx = base + j  ->  load l = idx / G, head idx % G, token l*TPL + lane/R
+    float sc[NF];
+    int hd[NF];
+    bool any_up = false;
+#pragma unroll
+    for (int j = 0; j < NF; ++j) {
+      const int idx = base + j;
+      const int tok = (idx / G) * TPL + lane / R;
+      const int t = chunk_t0 + tok;
+      const bool vis = stage_ok && t >= lo && t < L;
+      hd[j] = idx % G;
+      sc[j] = vis ? part[j] : -INFINITY;
+      float mr = m_ref[0];
+#pragma unroll
+      for (int hh = 1; hh < G; ++hh) mr = (hd[j] == hh) ? m_ref[hh] : mr;
+      any_up |= sc[j] > mr + kTau;
+    }
+    if (__any_sync(0xffffffffu, any_up)) {
+      // move the reference maxima to the new per-head maxima of this chunk
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) {
+        float mx = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < NF; ++j) mx = (hd[j] == hh) ? fmaxf(mx, sc[j]) : mx;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (mx > m_ref[hh] + kTau) {
+          const float alpha = (m_ref[hh] == -INFINITY) ? 0.f : ex2(m_ref[hh] - mx);
+          l_part[hh] *= alpha;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[hh][e] *= alpha;
+          m_ref[hh] = mx;
+        }
+      }
+    }
+    // probabilities relative to the reference maxima, shared through shared memory
+    float* pb = sm.pbuf[warp];
+#pragma unroll
+    for (int j = 0; j < NF; ++j) {
+      float mr = m_ref[0];
+#pragma unroll
+      for (int hh = 1; hh < G; ++hh) mr = (hd[j] == hh) ? m_ref[hh] : mr;
+      const float pr = (sc[j] == -INFINITY) ? 0.f : ex2(sc[j] - mr);
+      // with fewer values than lanes, DUP neighbouring lanes hold the same score: count it once
+      const bool counted = (lane & (DUP - 1)) == 0;
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) l_part[hh] += (hd[j] == hh && counted) ? pr : 0.f;
+      const int idx = base + j;
+      pb[((idx / G) * TPL + lane / R) * G + (idx % G)] = pr;
+    }
+    __syncwarp();
+
+    // ---- P.V over my 8 columns and my tokens
+#pragma unroll
+    for (int l = 0; l < NL; ++l) {
+      const int tok = l * TPL + lane / R;
+      uint4 u = sv[l * 32 + lane];
+      if (!full) {
+        const int t = chunk_t0 + tok;
+        if (!(stage_ok && t >= lo && t < L)) u = make_uint4(0u, 0u, 0u, 0u);  // poisoned slots stay out
+      }
+      float vf[8];
+      bf16x8_to_f32(u, vf);
+      float pv[G];
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) pv[hh] = pb[tok * G + hh];
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[hh][e] = fmaf(pv[hh], vf[e], acc[hh][e]);
+    }
+    __syncwarp();
+    fence_proxy_async_smem();
+    if (i + STAGES < n_my) issue(i + STAGES);
+  }
+
+  // ---- per-warp totals: accumulators over the TPL token groups, sums over all lanes
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh) {
+#pragma unroll
+    for (int o = R; o < 32; o <<= 1)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[hh][e] += __shfl_xor_sync(0xffffffffu, acc[hh][e], o);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l_part[hh] += __shfl_xor_sync(0xffffffffu, l_part[hh], o);
+  }
+  if (!ok_all) {
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) m_ref[hh] = -INFINITY;   // contribute nothing
+  }
+  // every stage this warp issued has been waited on, so the ring can be reused
+  __syncthreads();
+  float* wacc = reinterpret_cast<float*>(&sm.ring[0][0][0][0]);   // [kWarps][G][D]
+  if (lane < R) {
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) wacc[(warp * G + hh) * D + d0 + e] = acc[hh][e];
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) {
+      sm.wm[warp][hh] = m_ref[hh];
+      sm.wl[warp][hh] = l_part[hh];
+    }
+  }
+  __syncthreads();
+
+  // ---- merge the warps and write this split's partial output and lse
+  for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+    const int hh = idx / D, d = idx % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sm.wm[w][hh]);
+    float o = 0.f, lsum = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const float f = (sm.wm[w][hh] == -INFINITY) ? 0.f : ex2(sm.wm[w][hh] - M);
+        o += f * wacc[(w * G + hh) * D + d];
+        lsum += f * sm.wl[w][hh];
+      }
+    }
+    const size_t row = (static_cast<size_t>(b) * p.Hq + g * G + hh) * p.max_splits + s;
+    p.ws_o[row * D + d] = (lsum > 0.f) ? o / lsum : 0.f;
+    if (d == 0) p.ws_lse[row] = (lsum > 0.f) ? M + log2f(lsum) : -INFINITY;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams p, int N) {
+  constexpr int PER = D / 32;
+  const int warp_global = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (warp_global >= N * p.Hq) return;
+  const int b = warp_global / p.Hq;
+  int L = p.seq_lens[b];
+  L = min(L, min(p.max_seq_len, p.max_pages * p.page_size));
+  __nv_bfloat16* op = p.out + static_cast<size_t>(warp_global) * D;
+  float acc[PER];
+#pragma unroll
+  for (int t = 0; t < PER; ++t) acc[t] = 0.f;
+  float wsum = 0.f;
+  if (L > 0) {
+    const int lo = (p.window > 0) ? max(0, L - p.window) : 0;
+    const int s0 = lo / p.split_tokens, s1 = (L - 1) / p.split_tokens;
+    const size_t rowbase = static_cast<size_t>(warp_global) * p.max_splits;
+    float M = -INFINITY;
+    for (int s = s0; s <= s1; ++s) M = fmaxf(M, p.ws_lse[rowbase + s]);
+    if (M != -INFINITY) {
+      for (int s = s0; s <= s1; ++s) {
+        const float lse = p.ws_lse[rowbase + s];
+        const float w = (lse == -INFINITY) ? 0.f : ex2(lse - M);
+        wsum += w;
+        const float* o = p.ws_o + (rowbase + s) * D;
+#pragma unroll
+        for (int t = 0; t < PER; ++t) acc[t] = fmaf(w, o[lane * PER + t], acc[t]);
+      }
+    }
+  }
+  const float inv = (wsum > 0.f) ? 1.f / wsum : 0.f;
+#pragma unroll
+  for (int t = 0; t < PER; t += 2) {
+    __nv_bfloat162 v2 = __floats2bfloat162_rn(acc[t] * inv, acc[t + 1] * inv);
+    *reinterpret_cast<__nv_bfloat162*>(op + lane * PER + t) = v2;
+  }
+}
+
+template <int D, int G>
+cudaError_t launch_split(const DecodeParams& p, int N, cudaStream_t stream) {
+  const size_t smem = sizeof(SplitSmem<D, G>) + 1024;
+  auto kern = decode_split_kernel<D, G>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.max_splits, p.Hkv, N);
+  kern<<<grid, kWarps * 32, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+DecodeGeometry decode_geometry(int N, int Hq, int D, int max_seq_len, int page_size) {
+  (void)Hq;
+  (void)D;
+  (void)page_size;
+  DecodeGeometry g{};
+  // 512 keys per split: 8 chunks per warp, enough to amortise the pipeline
+  // fill; shorter splits when the batch is too small to fill the GPU.
+  int split = 512;
+  const long long units = static_cast<long long>(N);
+  while (split > 64 && units * ((max_seq_len + split - 1) / split) < 1024) split /= 2;
+  g.split_tokens = split;
+  g.max_splits = max_seq_len > 0 ? (max_seq_len + split - 1) / split : 1;
+  return g;
+}
+
+size_t decode_workspace_bytes(int N, int Hq, int D, int max_seq_len, int page_size) {
+  const DecodeGeometry g = decode_geometry(N, Hq, D, max_seq_len, page_size);
+  const size_t rows = static_cast<size_t>(N) * Hq * g.max_splits;
+  const size_t o_bytes = rows * D * sizeof(float);
+  const size_t lse_bytes = ((rows * sizeof(float)) + 255) & ~static_cast<size_t>(255);
+  return o_bytes + lse_bytes;
+}
+
+cudaError_t launch_decode_paged(const void* q, const void* k_pool, const void* v_pool, const int32_t* page_table,
+                                const int32_t* seq_lens, int page_size, int N, int Hq, int Hkv, int D,
+                                int num_pages, int max_pages, int max_seq_len, float scale, int window,
+                                void* workspace, void* out, unsigned int* err, cudaStream_t stream) {
+  const DecodeGeometry geo = decode_geometry(N, Hq, D, max_seq_len, page_size);
+  DecodeParams p{};
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k_pool = static_cast<const __nv_bfloat16*>(k_pool);
+  p.v_pool = static_cast<const __nv_bfloat16*>(v_pool);
+  p.page_table = page_table;
+  p.seq_lens = seq_lens;
+  const size_t rows = static_cast<size_t>(N) * Hq * geo.max_splits;
+  p.ws_o = static_cast<float*>(workspace);
+  p.ws_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + rows * D * sizeof(float));
+  p.err = err;
+  p.page_size = page_size;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.num_pages = num_pages;
+  p.max_pages = max_pages;
+  p.max_seq_len = max_seq_len;
+  p.split_tokens = geo.split_tokens;
+  p.max_splits = geo.max_splits;
+  p.window = window;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  const int G = Hq / Hkv;
+  cudaError_t e = cudaErrorInvalidValue;
+#define ATTN_DECODE_CASE(DD, GG) \
+  if (D == DD && G == GG) e = launch_split<DD, GG>(p, N, stream);
+  ATTN_DECODE_CASE(128, 1) ATTN_DECODE_CASE(128, 2) ATTN_DECODE_CASE(128, 4) ATTN_DECODE_CASE(128, 8)
+  ATTN_DECODE_CASE(64, 1) ATTN_DECODE_CASE(64, 2) ATTN_DECODE_CASE(64, 4) ATTN_DECODE_CASE(64, 8)
+#undef ATTN_DECODE_CASE
+  if (e != cudaSuccess) return e;
+  const int warps = N * Hq;
+  if (D == 128) {
+    decode_combine_kernel<128><<<(warps + 3) / 4, 128, 0, stream>>>(p, N);
+  } else {
+    decode_combine_kernel<64><<<(warps + 3) / 4, 128, 0, stream>>>(p, N);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace attn

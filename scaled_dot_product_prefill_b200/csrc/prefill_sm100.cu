@@ -1,0 +1,453 @@
+// prefill_sm100.cu -- bf16 attention prefill on the fifth-generation tensor cores.
+//
+// What is computed: O = softmax(Q K^T * scale + mask) V per (batch, query
+// head), with the causal / sliding-window masks and the GQA head map of the
+// public header.  The n x n score matrix is never written to memory: keys
+// are visited a tile at a time and an online softmax (running row maximum
+// and sum; earlier partial results rescaled when the maximum grows) gives
+// exactly the softmax of the full row ("Attention From Scratch" README,
+// section "Flash Attention"; "Taking LLMs apart (2)", section
+// "FlashAttention"; "Attention mechanism explained", section 7).
+//
+// How (one CTA = 2 query tiles x 128 rows of one head, 10 warps):
+//   warps 0-3  softmax group 0: thread t owns row t of query tile 0
+//   warps 4-7  softmax group 1: the same for query tile 1
+//   warp 8     TMA producer: Q once, then K_j / V_j tiles into a ring of
+//              shared-memory slots (128-byte swizzle, no multicast)
+//   warp 9     MMA issuer (one thread) and tensor-memory owner
+// Tensor memory (512 columns x 128 lanes, fp32):
+//   S_i = Q_i K_j^T   columns [128 i, 128 i + 128)      (tcgen05.mma, A and B in smem)
+//   P_i (bf16)        written over the first 64 columns of S_i by the softmax threads
+//   O_i += P_i V_j    columns [256 + D i, 256 + D i + D) (tcgen05.mma, A = P in tmem)
+// Per key tile j the MMA thread issues S_0, S_1 (K_j), then, as each
+// softmax group hands back P_i, the P_i V_j product.  Tensor-core work is
+// in order, so the commit that signals S_i(j) also guarantees that
+// P_i V_{j-1} has landed in O_i; the softmax thread may then rescale O_i.
+// The reference maximum only moves when a score exceeds it by 2^8 (in
+// probability), so the O rescale is rare after the first tiles and the
+// result stays exact.  Key tiles that the mask hides from every row of a
+// query tile are never loaded or multiplied; element masks are applied only
+// on tiles that straddle a mask edge.
+#include <cmath>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <mutex>
+
+#include "common.cuh"
+#include "sm100_ptx.cuh"
+
+namespace attn {
+namespace {
+
+constexpr int BM = 128;          // query rows per tile
+constexpr int BN = 128;          // keys per tile
+constexpr int NQ = 2;            // query tiles per CTA
+constexpr int kThreads = 320;    // 10 warps
+constexpr int kTmaWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kTau = 8.0f;     // lazy-rescale threshold, log2 units
+
+template <int D>
+struct Cfg {
+  static constexpr int KATOMS = D / 64;               // 64-column (128-byte) swizzle atoms
+  static constexpr int TILE_BYTES = BN * D * 2;       // one K or V tile
+  static constexpr int Q_BYTES = BM * D * 2;          // one query tile
+  static constexpr int STAGES = (D == 128) ? 4 : 6;   // ring slots; K and V tiles alternate
+  static constexpr uint32_t S_COL = 0;                // + 128 * i
+  static constexpr uint32_t O_COL = 256;              // + D * i
+  static constexpr size_t SMEM = 1024 /*align*/ + NQ * Q_BYTES + STAGES * TILE_BYTES + 256;
+};
+
+struct Params {
+  int B, Hq, Hkv, Sq, Skv, causal, window, n_qblocks;
+  float scale_log2;
+  __nv_bfloat16* out;
+  unsigned int* err;
+};
+
+struct Ranges {
+  int lo[NQ], hi[NQ];   // key-tile range per query tile (empty if hi <= lo)
+  int lo_all, hi_all;
+};
+
+__device__ __forceinline__ Ranges key_tile_ranges(const Params& p, int q_row0) {
+  Ranges R;
+  const int off = p.Skv - p.Sq;
+  const int n_kt = (p.Skv + BN - 1) / BN;
+  R.lo_all = 1 << 30;
+  R.hi_all = 0;
+#pragma unroll
+  for (int i = 0; i < NQ; ++i) {
+    const int r0 = q_row0 + BM * i;
+    const int r1 = min(r0 + BM, p.Sq);   // exclusive
+    int lo = 0, hi = 0;
+    if (r0 < p.Sq) {
+      if (!p.causal) {
+        lo = 0;
+        hi = n_kt;
+      } else {
+        const int last_key = min(r1 - 1 + off, p.Skv - 1);
+        const int first_key = (p.window > 0) ? max(0, r0 + off - p.window + 1) : 0;
+        if (last_key >= first_key && last_key >= 0) {
+          lo = first_key / BN;
+          hi = last_key / BN + 1;
+        }
+      }
+    }
+    R.lo[i] = lo;
+    R.hi[i] = hi;
+    if (hi > lo) {
+      R.lo_all = min(R.lo_all, lo);
+      R.hi_all = max(R.hi_all, hi);
+    }
+  }
+  if (R.hi_all <= 0) R.lo_all = R.hi_all = 0;
+  return R;
+}
+
+// True if every (row, key) pair of query tile rows [r0, r0+BM) x key tile j is visible.
+__device__ __forceinline__ bool tile_unmasked(const Params& p, int r0, int j) {
+  const int off = p.Skv - p.Sq;
+  const int k0 = j * BN, k1 = j * BN + BN - 1;
+  if (k1 >= p.Skv) return false;
+  if (!p.causal) return true;
+  if (k1 > r0 + off) return false;
+  if (p.window > 0 && k0 <= r0 + BM - 1 + off - p.window) return false;
+  return true;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                      const __grid_constant__ CUtensorMap tmap_v, const Params p) {
+  using C = Cfg<D>;
+  constexpr int STAGES = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem;                                   // [NQ][KATOMS][BM rows x 128 B]
+  uint8_t* sRing = smem + NQ * C::Q_BYTES;              // [STAGES][KATOMS][BN rows x 128 B]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sRing + STAGES * C::TILE_BYTES);
+  uint64_t* q_full = bars;                              // 1
+  uint64_t* full = bars + 1;                            // STAGES
+  uint64_t* empty = full + STAGES;                      // STAGES
+  uint64_t* s_ready = empty + STAGES;                   // NQ
+  uint64_t* p_ready = s_ready + NQ;                     // NQ
+  uint64_t* o_done = p_ready + NQ;                      // NQ
+  uint64_t* drain = o_done + NQ;                        // 1
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // heaviest query blocks first: block-major over (b, h) for the last query block, ...
+  const int BH = p.B * p.Hq;
+  const int bh = blockIdx.x % BH;
+  const int qb = p.n_qblocks - 1 - static_cast<int>(blockIdx.x / BH);
+  const int b = bh / p.Hq, h = bh % p.Hq;
+  const int g = h / (p.Hq / p.Hkv);
+  const int q_row0 = qb * (NQ * BM);
+  const Ranges R = key_tile_ranges(p, q_row0);
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < NQ; ++i) {
+      mbar_init(&s_ready[i], 1);
+      mbar_init(&p_ready[i], 4 * 32);
+      mbar_init(&o_done[i], 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kTmaWarp) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && R.hi_all > R.lo_all) {
+      prefetch_tmap(&tmap_q);
+      prefetch_tmap(&tmap_k);
+      prefetch_tmap(&tmap_v);
+      mbar_arrive_expect_tx(q_full, NQ * C::Q_BYTES);
+      for (int i = 0; i < NQ; ++i)
+        for (int a = 0; a < C::KATOMS; ++a)
+          tma_load_3d(sQ + (i * C::KATOMS + a) * BM * 128, &tmap_q, q_full, a * 64, q_row0 + BM * i, bh);
+      const int kv_plane = b * p.Hkv + g;
+      int n = 0;
+      bool ok = true;
+      for (int j = R.lo_all; j < R.hi_all && ok; ++j) {
+        for (int kv = 0; kv < 2 && ok; ++kv, ++n) {
+          const int st = n % STAGES;
+          if (!mbar_wait(&empty[st], ((n / STAGES) & 1) ^ 1, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[st], C::TILE_BYTES);
+          const CUtensorMap* tm = kv ? &tmap_v : &tmap_k;
+          for (int a = 0; a < C::KATOMS; ++a)
+            tma_load_3d(sRing + st * C::TILE_BYTES + a * BN * 128, tm, &full[st], a * 64, j * BN, kv_plane);
+        }
+      }
+      // the last loads issued must land before the CTA may exit (normally already consumed)
+      for (int k = max(0, n - STAGES); k < n; ++k) mbar_wait(&full[k % STAGES], (k / STAGES) & 1, nullptr, p.err);
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && R.hi_all > R.lo_all) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(BM, BN, 0, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, 0, 1);
+      const uint32_t q_addr = smem_u32(sQ);
+      const uint32_t ring_addr = smem_u32(sRing);
+      int n = 0;
+      int t[NQ] = {0, 0};
+      bool ok = mbar_wait(q_full, 0, abort_flag, p.err);
+      tc_fence_after();
+      for (int j = R.lo_all; j < R.hi_all && ok; ++j) {
+        // ---- S_i = Q_i K_j^T
+        int st = n % STAGES;
+        if (!(ok = mbar_wait(&full[st], (n / STAGES) & 1, abort_flag, p.err))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int i = 0; i < NQ; ++i) {
+          if (j < R.lo[i] || j >= R.hi[i]) continue;
+          const uint32_t d_tmem = tmem + C::S_COL + 128 * i;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t koff = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+            const uint64_t adesc = sw128_desc(q_addr + i * C::Q_BYTES + koff, 16, 1024);
+            const uint64_t bdesc = sw128_desc(ring_addr + st * C::TILE_BYTES + koff, 16, 1024);
+            mma_ss(d_tmem, adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&s_ready[i]);
+        }
+        mma_commit(&empty[st]);
+        ++n;
+        // ---- O_i += P_i V_j
+        st = n % STAGES;
+        if (!(ok = mbar_wait(&full[st], (n / STAGES) & 1, abort_flag, p.err))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int i = 0; i < NQ; ++i) {
+          if (j < R.lo[i] || j >= R.hi[i]) continue;
+          if (!(ok = mbar_wait(&p_ready[i], t[i] & 1, abort_flag, p.err))) break;
+          tc_fence_after();
+          const uint32_t o_tmem = tmem + C::O_COL + D * i;
+          const uint32_t p_tmem = tmem + C::S_COL + 128 * i;
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            const uint64_t bdesc = sw128_desc(ring_addr + st * C::TILE_BYTES + kk * 16 * 128, BN * 128, 1024);
+            mma_ts(o_tmem, p_tmem + kk * 8, bdesc, idesc_pv, (j > R.lo[i] || kk > 0) ? 1u : 0u);
+          }
+          ++t[i];
+        }
+        if (!ok) break;
+        mma_commit(&empty[st]);
+        ++n;
+#pragma unroll
+        for (int i = 0; i < NQ; ++i)
+          if (j == R.hi[i] - 1) mma_commit(&o_done[i]);
+      }
+      // everything issued above must be complete before tensor memory is released
+      mma_commit(drain);
+      mbar_wait(drain, 0, nullptr, p.err);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax groups
+    const int i = warp >> 2;                 // query tile
+    const int wq = warp & 3;                 // lane quarter of tensor memory
+    const int rl = wq * 32 + lane;           // row within the tile
+    const int r = q_row0 + BM * i + rl;      // query row
+    const int off = p.Skv - p.Sq;
+    const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t s_tmem = tmem + lane_bits + C::S_COL + 128 * i;
+    const uint32_t o_tmem = tmem + lane_bits + C::O_COL + D * i;
+    // visible keys of this row: [key_lo, key_hi]
+    const int key_hi = p.causal ? min(r + off, p.Skv - 1) : p.Skv - 1;
+    const int key_lo = (p.causal && p.window > 0) ? r + off - p.window + 1 : 0;
+    const int my_lo = (i == 0) ? R.lo[0] : R.lo[1];
+    const int my_hi = (i == 0) ? R.hi[0] : R.hi[1];
+    const bool have_keys = my_hi > my_lo;
+
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = my_lo, t = 0; j < my_hi; ++j, ++t) {
+      ok = mbar_wait(&s_ready[i], t & 1, abort_flag, p.err);
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[BN];
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c) tmem_ld32(s_tmem + 32 * c, sr + 32 * c);
+      tmem_wait_ld();
+      float s[BN];
+#pragma unroll
+      for (int c = 0; c < BN; ++c) s[c] = __uint_as_float(sr[c]);
+      if (!tile_unmasked(p, q_row0 + BM * i, j)) {
+        const int c_lo = key_lo - j * BN, c_hi = key_hi - j * BN;
+#pragma unroll
+        for (int c = 0; c < BN; ++c) s[c] = (c >= c_lo && c <= c_hi) ? s[c] : -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
+      const float m_tile = mx * p.scale_log2;
+      float alpha = 1.f;
+      if (m_tile > m_ref + kTau) {
+        alpha = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - m_tile);
+        l *= alpha;
+        m_ref = m_tile;
+      }
+      const bool rescale = (t > 0) && (alpha != 1.f);
+      if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(o_tmem + 32 * c, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(o_tmem + 32 * c, o);
+        }
+      }
+      const float mb = (m_ref == -INFINITY) ? 0.f : m_ref;
+      uint32_t pk[BN / 2];
+      float lsum = 0.f;
+#pragma unroll
+      for (int c = 0; c < BN; c += 2) {
+        const float p0 = ex2(fmaf(s[c], p.scale_log2, -mb));
+        const float p1 = ex2(fmaf(s[c + 1], p.scale_log2, -mb));
+        lsum += p0 + p1;
+        pk[c / 2] = pack_bf16x2(p0, p1);
+      }
+      l += lsum;
+#pragma unroll
+      for (int c = 0; c < BN / 64; ++c)
+        tmem_st32(s_tmem + 32 * c, pk + 32 * c);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_ready[i]);
+    }
+    // ---- epilogue: O / l -> bf16
+    if (ok && have_keys) {
+      ok = mbar_wait(&o_done[i], 0, abort_flag, p.err);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok && r < p.Sq) {
+      __nv_bfloat16* orow = p.out + (static_cast<size_t>(bh) * p.Sq + r) * D;
+      if (have_keys) {
+        tc_fence_after();
+        const float inv = (l > 0.f) ? 1.f / l : 0.f;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(o_tmem + 32 * c, o);
+          tmem_wait_ld();
+          uint4 pk4[4];
+          uint32_t* pk = reinterpret_cast<uint32_t*>(pk4);
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dst[e] = pk4[e];
+        }
+      } else {
+        uint4* dst = reinterpret_cast<uint4*>(orow);
+        for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    } else if (!ok && have_keys) {
+      // a wait gave up: the rows stay unwritten; the error word says so
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn tensor_map_encoder() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// [planes][rows][D] bf16 tensor, boxes of 64 columns x 128 rows, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int D, int rows, int planes) {
+  EncodeTiledFn enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(planes)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(rows) * D * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t launch_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const Params& p,
+                     cudaStream_t stream) {
+  auto kern = prefill_tc_kernel<D>;
+  const size_t smem = Cfg<D>::SMEM;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>(p.n_qblocks) * static_cast<unsigned>(p.B * p.Hq);
+  kern<<<grid, kThreads, smem, stream>>>(mq, mk, mv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv,
+                              int Sq, int Skv, int D, float scale, int causal, int window, unsigned int* err,
+                              cudaStream_t stream) {
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, D, Sq, B * Hq) || !make_map(&mk, k, D, Skv, B * Hkv) || !make_map(&mv, v, D, Skv, B * Hkv))
+    return cudaErrorInvalidValue;
+  Params p{};
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Sq = Sq;
+  p.Skv = Skv;
+  p.causal = causal;
+  p.window = window;
+  p.n_qblocks = (Sq + NQ * BM - 1) / (NQ * BM);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.err = err;
+  return D == 64 ? launch_d<64>(mq, mk, mv, p, stream) : launch_d<128>(mq, mk, mv, p, stream);
+}
+
+}  // namespace attn

@@ -32,3 +32,26 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch.device("cuda:0")
+
+
+# bf16 configurations: max-abs <= 2e-2 and mean-abs <= 2e-3 against the float64 oracle;
+# fp32 configuration: max-abs <= 1e-4.
+BF16_MAX_ABS, BF16_MEAN_ABS = 2e-2, 2e-3
+F32_MAX_ABS = 1e-4
+
+
+def assert_parity(got, ref, dtype="bf16", what=""):
+    """Element-by-element comparison of a GPU result with the float64 oracle."""
+    import numpy as np
+
+    g = got.detach().to("cpu").double().numpy() if hasattr(got, "detach") else np.asarray(got, dtype=np.float64)
+    r = np.asarray(ref, dtype=np.float64)
+    assert g.shape == r.shape, (g.shape, r.shape)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite output"
+    err = np.abs(g - r)
+    mx, mean = float(err.max()) if err.size else 0.0, float(err.mean()) if err.size else 0.0
+    if dtype == "bf16":
+        assert mx <= BF16_MAX_ABS and mean <= BF16_MEAN_ABS, f"{what}: max-abs {mx:.3e} mean-abs {mean:.3e}"
+    else:
+        assert mx <= F32_MAX_ABS, f"{what}: max-abs {mx:.3e}"
+    return mx, mean

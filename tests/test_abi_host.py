@@ -1,0 +1,125 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared
+entry point, and rejects bad arguments before touching the GPU.  CPU only."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "attn_b200.h")
+
+
+def _lib():
+    from scaled_dot_product_prefill_b200 import _lib
+
+    if not os.path.exists(_lib.lib_path()):
+        from scaled_dot_product_prefill_b200 import build
+
+        build.build()
+    return _lib.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("attn_prefill", "attn_prefill_f32", "attn_decode_paged",
+                     "attn_decode_paged_workspace_size", "attn_status_string", "attn_device_status"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib()
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in attn_b200.h but not exported"
+
+
+def test_binding_prototypes_cover_the_header():
+    from scaled_dot_product_prefill_b200 import _lib as L
+
+    assert set(declared_functions()) == set(L.PROTOTYPES)
+
+
+def test_status_strings_and_version():
+    lib = _lib()
+    assert lib.attn_status_string(0) == b"ATTN_OK"
+    assert lib.attn_status_string(6) == b"ATTN_ERR_WORKSPACE"
+    assert lib.attn_status_string(99) == b"ATTN_ERR_UNKNOWN"
+    assert lib.attn_version() >= 100
+
+
+FAKE = ctypes.c_void_p(0x10000)          # aligned, never dereferenced: every case below fails validation
+MISALIGNED = ctypes.c_void_p(0x10008)
+
+
+def prefill(lib, fn="attn_prefill", q=FAKE, k=FAKE, v=FAKE, o=FAKE, B=1, Hq=4, Hkv=2, Sq=64, Skv=64, D=64,
+            scale=0.125, causal=1, window=0):
+    return getattr(lib, fn)(q, k, v, o, B, Hq, Hkv, Sq, Skv, D, scale, causal, window, None)
+
+
+@pytest.mark.parametrize("fn", ["attn_prefill", "attn_prefill_f32"])
+def test_prefill_argument_validation(fn):
+    lib = _lib()
+    assert prefill(lib, fn, q=None) == 1
+    assert prefill(lib, fn, o=MISALIGNED) == 1
+    assert prefill(lib, fn, Hq=6, Hkv=4) == 1           # Hq not a multiple of Hkv
+    assert prefill(lib, fn, Hkv=0) == 1
+    assert prefill(lib, fn, Sq=-1) == 1
+    assert prefill(lib, fn, scale=0.0) == 1
+    assert prefill(lib, fn, scale=float("nan")) == 1
+    assert prefill(lib, fn, causal=2) == 1
+    assert prefill(lib, fn, window=-3) == 1
+    assert prefill(lib, fn, D=96) == 2                  # head dim not implemented
+    assert prefill(lib, fn, causal=0, window=16) == 2   # a window is a causal look-back
+    # empty problems are no-ops, even with null pointers
+    assert prefill(lib, fn, q=None, k=None, v=None, o=None, B=0) == 0
+    assert prefill(lib, fn, q=None, k=None, v=None, o=None, Sq=0) == 0
+
+
+def decode(lib, q=FAKE, kp=FAKE, vp=FAKE, pt=FAKE, sl=FAKE, page=16, N=4, Hq=8, Hkv=2, D=128, num_pages=64,
+           max_pages=16, max_seq_len=256, scale=0.1, window=0, ws=FAKE, ws_bytes=1 << 30, out=FAKE):
+    return lib.attn_decode_paged(q, kp, vp, pt, sl, page, N, Hq, Hkv, D, num_pages, max_pages, max_seq_len,
+                                 scale, window, ws, ws_bytes, out, None)
+
+
+def test_decode_argument_validation():
+    lib = _lib()
+    assert decode(lib, q=None) == 1
+    assert decode(lib, kp=None) == 1
+    assert decode(lib, Hq=8, Hkv=3) == 1
+    assert decode(lib, kp=MISALIGNED) == 1
+    assert decode(lib, scale=-1.0) == 1
+    assert decode(lib, D=96) == 2
+    assert decode(lib, Hq=24, Hkv=2) == 2               # group of 12
+    assert decode(lib, page=8) == 2
+    assert decode(lib, ws=None) == 6
+    need = lib.attn_decode_paged_workspace_size(4, 8, 128, 256, 16)
+    assert need > 0
+    assert decode(lib, ws_bytes=need - 1) == 6
+    assert decode(lib, N=0, q=None, out=None) == 0
+
+
+def test_workspace_size_is_monotone_and_rejects_bad_sizes():
+    lib = _lib()
+    a = lib.attn_decode_paged_workspace_size(64, 32, 128, 8192, 16)
+    b = lib.attn_decode_paged_workspace_size(64, 32, 128, 16384, 16)
+    assert 0 < a < b
+    assert lib.attn_decode_paged_workspace_size(-1, 32, 128, 8192, 16) == 0
+    # partial outputs and log-sum-exps: N * Hq * splits * (D + 1) floats, at most one split per 64 keys
+    assert a >= 64 * 32 * (8192 // 512) * 129 * 4
+
+
+def test_oracle_is_not_imported_by_the_library():
+    import sys
+
+    for mod in [m for m in list(sys.modules) if m.startswith("scaled_dot_product_prefill_b200")]:
+        src = getattr(sys.modules[mod], "__file__", None)
+        if src and src.endswith(".py"):
+            text = open(src).read()
+            assert "import oracle" not in text and "from oracle" not in text, src

@@ -1,0 +1,141 @@
+"""GPU parity of the prefill kernels against the float64 oracle (needs a B200).
+
+Small shapes are compared element by element on every output; the
+full-size workloads run in the launch configuration the benchmark times and
+are compared on sampled rows that the oracle evaluates one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+from conftest import assert_parity
+from oracle import sdpa
+from scaled_dot_product_prefill_b200 import api, inputs, workloads
+
+pytestmark = pytest.mark.gpu
+
+
+def run_prefill(inp, causal, window, scale=None, dtype="bf16"):
+    q, k, v = (t.cuda() for t in (inp.q, inp.k, inp.v))
+    fn = api.attn_prefill if dtype == "bf16" else api.attn_prefill_f32
+    out = fn(q, k, v, causal=causal, window=window, scale=scale)
+    torch.cuda.synchronize()
+    assert api.attn_device_status(clear=True) == 0
+    return out
+
+
+SMALL = [
+    # B, Hq, Hkv, Sq, Skv, D, causal, window
+    (1, 1, 1, 1, 1, 64, False, 0),
+    (1, 2, 2, 17, 17, 64, True, 0),           # shorter than one tile
+    (2, 4, 2, 300, 300, 128, True, 0),        # ragged tail, GQA
+    (1, 4, 1, 300, 300, 64, False, 0),        # MQA, non-causal, ragged keys
+    (1, 2, 2, 600, 600, 128, True, 0),        # several query blocks
+    (1, 2, 1, 200, 700, 128, True, 0),        # Sq < Skv: bottom-right causal (chunked prefill)
+    (1, 2, 2, 700, 200, 64, True, 0),         # Sq > Skv: leading rows see no key
+    (1, 2, 2, 520, 520, 128, True, 1),        # window 1: every row sees itself only
+    (1, 2, 2, 520, 520, 64, True, 129),       # window across tile edges
+    (1, 4, 2, 640, 640, 128, True, 5000),     # window wider than the sequence
+    (3, 8, 8, 256, 256, 64, True, 0),         # exactly one query block
+    (1, 8, 2, 384, 1000, 64, False, 0),
+]
+
+
+@pytest.mark.parametrize("shape", SMALL, ids=[str(s) for s in SMALL])
+def test_prefill_bf16_matches_oracle(shape):
+    B, Hq, Hkv, Sq, Skv, D, causal, window = shape
+    inp = inputs.prefill_inputs(B, Hq, Hkv, Sq, Skv, D, seed=hash(shape) % 10000)
+    out = run_prefill(inp, causal, window)
+    ref = sdpa.attention(inp.q, inp.k, inp.v, 1.0 / np.sqrt(D), causal, window)
+    assert_parity(out, ref, "bf16", str(shape))
+
+
+@pytest.mark.parametrize("shape", [(1, 1, 1, 256, 256, 64, False, 0), (2, 4, 2, 300, 300, 128, True, 0),
+                                   (1, 2, 2, 200, 333, 64, True, 50), (1, 2, 2, 90, 40, 64, True, 0)])
+def test_prefill_f32_matches_oracle(shape):
+    B, Hq, Hkv, Sq, Skv, D, causal, window = shape
+    inp = inputs.prefill_inputs(B, Hq, Hkv, Sq, Skv, D, seed=7, dtype="f32")
+    out = run_prefill(inp, causal, window, dtype="f32")
+    ref = sdpa.attention(inp.q, inp.k, inp.v, 1.0 / np.sqrt(D), causal, window)
+    assert_parity(out, ref, "f32", str(shape))
+
+
+def test_single_head_f32_workload():
+    spec = workloads.WORKLOADS["single_head_f32"]
+    inp = inputs.prefill_inputs(spec.B, spec.Hq, spec.Hkv, spec.Sq, spec.Skv, spec.D, spec.seed, "f32")
+    out = run_prefill(inp, spec.causal, spec.window, spec.scale, dtype="f32")
+    ref = sdpa.attention(inp.q, inp.k, inp.v, spec.scale, spec.causal, spec.window)
+    assert_parity(out, ref, "f32", spec.name)
+
+
+def test_gpt2_small_causal_workload_full():
+    spec = workloads.WORKLOADS["mha_causal_gpt2s"]
+    inp = inputs.prefill_inputs(spec.B, spec.Hq, spec.Hkv, spec.Sq, spec.Skv, spec.D, spec.seed)
+    out = run_prefill(inp, spec.causal, spec.window, spec.scale)
+    ref = sdpa.attention(inp.q, inp.k, inp.v, spec.scale, spec.causal, spec.window)
+    assert_parity(out, ref, "bf16", spec.name)
+
+
+def sampled_rows(Sq, rng, n=48):
+    edges = [0, 1, 127, 128, 255, 256, Sq - 129, Sq - 128, Sq - 1]
+    rows = set(r for r in edges if 0 <= r < Sq) | set(rng.integers(0, Sq, n).tolist())
+    return sorted(rows)
+
+
+@pytest.mark.parametrize("name", ["gqa_causal_4k", "gqa_swa_16k"])
+def test_large_workloads_on_sampled_rows(name):
+    spec = workloads.WORKLOADS[name]
+    inp = inputs.prefill_inputs(spec.B, spec.Hq, spec.Hkv, spec.Sq, spec.Skv, spec.D, spec.seed)
+    out = run_prefill(inp, spec.causal, spec.window, spec.scale).cpu()
+    rng = np.random.default_rng(spec.seed)
+    G = spec.Hq // spec.Hkv
+    heads = [(0, 0), (spec.B - 1, spec.Hq - 1), (0, G), (spec.B // 2, spec.Hq // 2 + 1)]
+    for b, h in heads:
+        rows = sampled_rows(spec.Sq, rng)
+        g = h // G
+        ref = sdpa.attention_rows(inp.q[b, h, rows], inp.k[b, g], inp.v[b, g], rows, spec.Sq, spec.scale,
+                                  spec.causal, spec.window)
+        assert_parity(out[b, h, rows], ref, "bf16", f"{name} b={b} h={h}")
+    # every output is finite and, being a convex combination of values, bounded by max |v|
+    assert torch.isfinite(out.float()).all()
+    assert out.float().abs().max() <= inp.v.float().abs().max() + 1e-2
+
+
+def test_future_perturbation_leaves_past_rows_unchanged():
+    inp = inputs.prefill_inputs(2, 4, 2, 700, 700, 128, seed=11)
+    base = run_prefill(inp, True, 0)
+    k2, v2 = inp.k.clone(), inp.v.clone()
+    k2[:, :, 333:] += 10.0
+    v2[:, :, 333:] -= 7.0
+    pert = inputs.PrefillInputs(inp.q, k2, v2, 0)
+    out2 = run_prefill(pert, True, 0)
+    assert torch.equal(base[:, :, :333], out2[:, :, :333])
+    assert not torch.equal(base[:, :, 333:], out2[:, :, 333:])
+
+
+def test_shift_invariance_on_gpu():
+    """Adding one vector to every key shifts each row's logits by a constant; outputs must not move."""
+    inp = inputs.prefill_inputs(1, 2, 2, 384, 384, 64, seed=5)
+    base = run_prefill(inp, True, 0).float()
+    u = torch.full((64,), 0.5).to(torch.bfloat16)
+    k2 = (inp.k.float() + u.float()).to(torch.bfloat16)
+    out2 = run_prefill(inputs.PrefillInputs(inp.q, k2, inp.v, 0), True, 0).float()
+    ref2 = sdpa.attention(inp.q, k2, inp.v, 0.125, True, 0)
+    assert_parity(out2, ref2, "bf16", "shifted keys")
+    assert (out2 - base).abs().max() < 2e-2
+
+
+def test_gqa_equals_mha_on_repeated_heads():
+    inp = inputs.prefill_inputs(1, 8, 2, 256, 256, 128, seed=9)
+    gqa = run_prefill(inp, True, 0)
+    rep = inputs.PrefillInputs(inp.q, inp.k.repeat_interleave(4, dim=1).contiguous(),
+                               inp.v.repeat_interleave(4, dim=1).contiguous(), 0)
+    mha = run_prefill(rep, True, 0)
+    assert torch.equal(gqa, mha)
+
+
+def test_repeated_calls_are_deterministic():
+    inp = inputs.prefill_inputs(2, 4, 4, 512, 512, 64, seed=3)
+    a = run_prefill(inp, True, 0)
+    b = run_prefill(inp, True, 0)
+    assert torch.equal(a, b)
