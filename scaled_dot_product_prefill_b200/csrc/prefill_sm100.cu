@@ -347,8 +347,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = mbar_wait(&o_done[i], 0, abort_flag, p.err);
       ok = __all_sync(0xffffffffu, ok);
     }
-    if (ok && r < p.Sq) {
+    // tcgen05.ld is warp-collective (.sync.aligned): every lane loads, only rows < Sq store
+    if (ok) {
       __nv_bfloat16* orow = p.out + (static_cast<size_t>(bh) * p.Sq + r) * D;
+      const bool store = r < p.Sq;
       if (have_keys) {
         tc_fence_after();
         const float inv = (l > 0.f) ? 1.f / l : 0.f;
@@ -362,17 +364,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e)
             pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+          if (store) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = pk4[e];
+            for (int e = 0; e < 4; ++e) dst[e] = pk4[e];
+          }
         }
-      } else {
+      } else if (store) {
         uint4* dst = reinterpret_cast<uint4*>(orow);
         for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
       }
-    } else if (!ok && have_keys) {
-      // a wait gave up: the rows stay unwritten; the error word says so
     }
+    // if a wait gave up, the rows stay unwritten and the error word records it
   }
 
   tc_fence_before();
