@@ -32,7 +32,8 @@
  * - Pointers named q, k, v, out, k_pool, v_pool, page_table, seq_lens and
  *   workspace are DEVICE pointers of the current CUDA device, 16-byte
  *   aligned, owned by the caller.  The library never allocates or frees
- *   device memory and keeps no state between calls (re-entrant).
+ *   device memory and keeps no state between calls (re-entrant; the one
+ *   exception, attn_decode_paged_noalloc, is described at its declaration).
  * - bf16 means IEEE bfloat16 stored in 16 bits; inputs are read as bf16,
  *   all arithmetic accumulates in fp32, outputs are rounded to bf16 with
  *   round-to-nearest-even.
@@ -160,6 +161,35 @@ attn_status_t attn_decode_paged(const void* q, const void* k_pool, const void* v
                                 float scale, int window,
                                 void* workspace, size_t workspace_bytes,
                                 void* out, attn_stream_t stream);
+
+/*
+ * attn_decode_paged_noalloc -- attn_decode_paged for callers that cannot
+ * allocate device memory: callers behind an interface with no workspace
+ * argument (a plugin ABI fixed by a host framework), or serving loops whose
+ * device memory is planned once at start-up, where a cudaMalloc (which may
+ * also synchronise the device) is not allowed at decode time.  The source
+ * pages have no counterpart; this is a deployment variant of the same call.
+ *
+ * Arguments, layouts and results are those of attn_decode_paged without the
+ * workspace pair.  The split partials live in a fixed 32 MiB array inside
+ * the library, which every GPU that loads the library holds until the
+ * process exits; the call allocates and frees nothing.
+ * - Sizes whose attn_decode_paged_workspace_size exceeds 32 MiB
+ *   (33554432 bytes) are rejected with ATTN_ERR_WORKSPACE before any launch.
+ * - The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ * - All calls share the array: calls that overlap on the GPU (other streams,
+ *   other host threads) race on it and must be serialised by the caller.
+ *   Nothing in it needs clearing between calls.
+ * Errors: as attn_decode_paged, plus ATTN_ERR_WORKSPACE for sizes over the
+ * limit and ATTN_ERR_CUDA if the address lookup fails.
+ */
+attn_status_t attn_decode_paged_noalloc(const void* q, const void* k_pool, const void* v_pool,
+                                        const int32_t* page_table, const int32_t* seq_lens,
+                                        int page_size, int N, int Hq, int Hkv, int D,
+                                        int num_pages, int max_pages, int max_seq_len,
+                                        float scale, int window, void* out, attn_stream_t stream);
 
 /* Bytes of workspace attn_decode_paged needs for these sizes (0 if any size
  * is invalid).  Pure host arithmetic, no CUDA call. */

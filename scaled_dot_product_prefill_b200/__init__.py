@@ -5,5 +5,6 @@ include/attn_b200.h); ``api`` marshals torch tensors into it.  Importing the
 package does not load the library; the first call does, and raises if the
 library has not been built.
 """
-from .api import (AttnError, attn_decode_paged, attn_decode_paged_workspace_size,  # noqa: F401
+from .api import (AttnError, attn_decode_paged, attn_decode_paged_noalloc,  # noqa: F401
+                  attn_decode_paged_workspace_size,
                   attn_device_status, attn_prefill, attn_prefill_f32, attn_status_string, attn_version)

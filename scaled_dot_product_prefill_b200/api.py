@@ -13,7 +13,8 @@ import torch
 from . import _lib
 from ._lib import AttnError
 
-__all__ = ["attn_prefill", "attn_prefill_f32", "attn_decode_paged", "attn_decode_paged_workspace_size",
+__all__ = ["attn_prefill", "attn_prefill_f32", "attn_decode_paged", "attn_decode_paged_noalloc",
+           "attn_decode_paged_workspace_size",
            "attn_device_status", "attn_status_string", "attn_version", "AttnError"]
 
 
@@ -106,6 +107,29 @@ def attn_decode_paged(q, k_pool, v_pool, page_table, seq_lens, *, max_seq_len, s
         _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(page_table), _ptr(seq_lens), page_size, N, Hq, Hkv, D,
         num_pages, max_pages, int(max_seq_len), float(scale), int(window), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(out), _stream(stream)))
+    return out
+
+
+def attn_decode_paged_noalloc(q, k_pool, v_pool, page_table, seq_lens, *, max_seq_len, scale=None, window=0,
+                              out=None, stream=None):
+    """attn_decode_paged with the library's fixed 32 MiB scratch instead of a workspace.
+
+    For callers that cannot allocate device memory when they decode.  Calls
+    that overlap on the GPU share (and race on) that scratch.
+    """
+    N, Hq, D = q.shape
+    num_pages, Hkv, page_size, _ = k_pool.shape
+    max_pages = page_table.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    _need_cuda(q, k_pool, v_pool, page_table, seq_lens, out)
+    if page_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise ValueError("page_table and seq_lens must be int32")
+    _check("attn_decode_paged_noalloc", _lib.load().attn_decode_paged_noalloc(
+        _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(page_table), _ptr(seq_lens), page_size, N, Hq, Hkv, D,
+        num_pages, max_pages, int(max_seq_len), float(scale), int(window), _ptr(out), _stream(stream)))
     return out
 
 

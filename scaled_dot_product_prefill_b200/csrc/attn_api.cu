@@ -128,6 +128,23 @@ attn_status_t attn_decode_paged(const void* q, const void* k_pool, const void* v
                                              attn::device_error_word(), reinterpret_cast<cudaStream_t>(stream)));
 }
 
+attn_status_t attn_decode_paged_noalloc(const void* q, const void* k_pool, const void* v_pool,
+                                        const int32_t* page_table, const int32_t* seq_lens, int page_size, int N,
+                                        int Hq, int Hkv, int D, int num_pages, int max_pages, int max_seq_len,
+                                        float scale, int window, void* out, attn_stream_t stream) {
+  // Same checks as attn_decode_paged, with the library's fixed scratch as the workspace.
+  if (N < 0 || Hq < 0 || D <= 0 || max_seq_len < 0 || page_size <= 0) return ATTN_ERR_INVALID_ARG;
+  const size_t need = (N == 0 || Hq == 0) ? 0 : attn::decode_workspace_bytes(N, Hq, D, max_seq_len, page_size);
+  if (need > attn::decode_scratch_capacity()) return ATTN_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if (need > 0) {
+    scratch = attn::decode_scratch_address();
+    if (scratch == nullptr) return ATTN_ERR_CUDA;
+  }
+  return attn_decode_paged(q, k_pool, v_pool, page_table, seq_lens, page_size, N, Hq, Hkv, D, num_pages, max_pages,
+                           max_seq_len, scale, window, scratch, attn::decode_scratch_capacity(), out, stream);
+}
+
 attn_status_t attn_device_status(int clear) {
   unsigned int* addr = attn::device_error_word();
   if (addr == nullptr) return ATTN_ERR_CUDA;

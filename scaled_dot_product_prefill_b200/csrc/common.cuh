@@ -38,6 +38,8 @@ struct DecodeGeometry {
 };
 DecodeGeometry decode_geometry(int N, int Hq, int D, int max_seq_len, int page_size);
 size_t decode_workspace_bytes(int N, int Hq, int D, int max_seq_len, int page_size);
+size_t decode_scratch_capacity();
+void* decode_scratch_address();
 cudaError_t launch_decode_paged(const void* q, const void* k_pool, const void* v_pool, const int32_t* page_table,
                                 const int32_t* seq_lens, int page_size, int N, int Hq, int Hkv, int D,
                                 int num_pages, int max_pages, int max_seq_len, float scale, int window,

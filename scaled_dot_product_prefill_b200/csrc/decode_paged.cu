@@ -32,6 +32,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <mutex>
 
 #include "common.cuh"
 #include "sm100_ptx.cuh"
@@ -481,6 +482,43 @@ cudaError_t launch_decode_paged(const void* q, const void* k_pool, const void* v
     decode_combine_kernel<64><<<(warps + 3) / 4, 128, 0, stream>>>(p, N);
   }
   return cudaGetLastError();
+}
+
+
+// ---------------------------------------------------------------------------
+// Fixed scratch for attn_decode_paged_noalloc.
+//
+// Some callers cannot allocate device memory at the point where they decode:
+// code behind an interface that has no workspace argument (a plugin ABI fixed
+// by a host framework), or a serving loop whose device memory is planned once
+// at start-up and where a cudaMalloc, which may also synchronise the device,
+// is not allowed.  For them the split-KV partials live in this file-scope
+// array instead of a caller-provided workspace.  Every GPU that loads the
+// library holds these kDecodeScratchBytes until the process exits.  All calls
+// share the array: calls that overlap on the GPU (two streams, or two
+// threads) race on it.  Nothing in it needs to start at zero: each call
+// writes every partial output and log-sum-exp it later reads.
+constexpr size_t kDecodeScratchBytes = size_t(32) << 20;   // 32 MiB
+static __device__ __align__(256) unsigned char g_decode_scratch[kDecodeScratchBytes];
+
+size_t decode_scratch_capacity() { return kDecodeScratchBytes; }
+
+// Device address of g_decode_scratch on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up with
+// cudaGetSymbolAddress, once per device, with that device current, and cached.
+void* decode_scratch_address() {
+  constexpr int kMaxDevices = 64;
+  static void* addr[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = ptr;
+  }
+  return addr[dev];
 }
 
 }  // namespace attn
