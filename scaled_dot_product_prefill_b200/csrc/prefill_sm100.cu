@@ -9,22 +9,27 @@
 // section "Flash Attention"; "Taking LLMs apart (2)", section
 // "FlashAttention"; "Attention mechanism explained", section 7).
 //
-// How (one CTA = 2 query tiles x 128 rows of one head, 10 warps):
+// How.  A work item is a block of 2 x 128 query rows of one (batch, head).
+// The kernel is persistent: one CTA per SM walks the items in order of
+// decreasing cost (later causal blocks first), dealt out in a snake so that
+// the SMs finish together.  Each CTA has 12 warps:
 //   warps 0-3  softmax group 0: thread t owns row t of query tile 0
 //   warps 4-7  softmax group 1: the same for query tile 1
-//   warp 8     TMA producer: Q once, then K_j / V_j tiles into a ring of
-//              shared-memory slots (128-byte swizzle, no multicast)
+//   warp 8     TMA producer: Q of each item, then K_j / V_j tiles into a ring
+//              of shared-memory slots (128-byte swizzle, no multicast)
 //   warp 9     MMA issuer (one thread) and tensor-memory owner
+//   warps 10-11 idle (complete the third warpgroup for the register split)
 // Tensor memory (512 columns x 128 lanes, fp32):
-//   S_i = Q_i K_j^T   columns [128 i, 128 i + 128)      (tcgen05.mma, A and B in smem)
-//   P_i (bf16)        written over the first 64 columns of S_i by the softmax threads
-//   O_i += P_i V_j    columns [256 + D i, 256 + D i + D) (tcgen05.mma, A = P in tmem)
-// Per key tile j the MMA thread issues S_0, S_1 (K_j), then, as each
-// softmax group hands back P_i, the P_i V_j product.  Tensor-core work is
-// in order, so the commit that signals S_i(j) also guarantees that
-// P_i V_{j-1} has landed in O_i; the softmax thread may then rescale O_i.
-// The reference maximum only moves when a score exceeds it by 2^8 (in
-// probability), so the O rescale is rare after the first tiles and the
+//   S_i = Q_i K_j^T   columns [128 i, 128 i + 128)      (A and B in smem)
+//   P_i (bf16)        written over the first 64 columns of S_i by the softmax
+//   O_i += P_i V_j    columns [256 + D i, 256 + D i + D) (A = P in tmem)
+// The MMA thread alternates the two query tiles: as soon as group i hands
+// back P_i(j) it issues P_i(j) V_j and then S_i(j+1), so one group's softmax
+// overlaps the other group's matrix products.  Tensor-core work is in
+// order, so the commit that signals S_i(j+1) also covers P_i(j) V_j: the
+// softmax thread may then rescale O_i without another barrier.  The
+// reference maximum only moves when a score exceeds it by 2^8 (in
+// probability), so rescaling is rare after the first key tile and the
 // result stays exact.  Key tiles that the mask hides from every row of a
 // query tile are never loaded or multiplied; element masks are applied only
 // on tiles that straddle a mask edge.
@@ -42,10 +47,17 @@ namespace {
 
 constexpr int BM = 128;          // query rows per tile
 constexpr int BN = 128;          // keys per tile
-constexpr int NQ = 2;            // query tiles per CTA
-constexpr int kThreads = 320;    // 10 warps
+constexpr int NQ = 2;            // query tiles per work item
+constexpr int kThreads = 384;    // 12 warps = 3 warpgroups
 constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;
+// Register split (setmaxnreg works per warpgroup): the two softmax groups hold
+// a 128-column score row each and get kSoftmaxRegs; the producer group (TMA
+// and MMA warps, two idle warps) gets kProducerRegs.  The split must fit the
+// launch allocation: 128 * (2 * kSoftmaxRegs + kProducerRegs) <= kThreads *
+// regs-per-thread at launch, which the host checks before every launch.
+constexpr int kSoftmaxRegs = 200;
+constexpr int kProducerRegs = 104;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kTau = 8.0f;     // lazy-rescale threshold, log2 units
 
@@ -54,38 +66,52 @@ struct Cfg {
   static constexpr int KATOMS = D / 64;               // 64-column (128-byte) swizzle atoms
   static constexpr int TILE_BYTES = BN * D * 2;       // one K or V tile
   static constexpr int Q_BYTES = BM * D * 2;          // one query tile
+  static constexpr int QBUF = (D == 128) ? 1 : 2;     // query buffers (items in flight)
   static constexpr int STAGES = (D == 128) ? 4 : 6;   // ring slots; K and V tiles alternate
   static constexpr uint32_t S_COL = 0;                // + 128 * i
   static constexpr uint32_t O_COL = 256;              // + D * i
-  static constexpr size_t SMEM = 1024 /*align*/ + NQ * Q_BYTES + STAGES * TILE_BYTES + 256;
+  static constexpr size_t SMEM = 1024 /*align*/ + QBUF * NQ * Q_BYTES + STAGES * TILE_BYTES + 256;
 };
 
 struct Params {
-  int B, Hq, Hkv, Sq, Skv, causal, window, n_qblocks;
+  int B, Hq, Hkv, Sq, Skv, causal, window, n_qblocks, n_items;
   float scale_log2;
   __nv_bfloat16* out;
   unsigned int* err;
 };
 
-struct Ranges {
+struct Item {
+  int bh, b, g, q_row0;
   int lo[NQ], hi[NQ];   // key-tile range per query tile (empty if hi <= lo)
-  int lo_all, hi_all;
+  int lo_all, hi_all;   // union; empty if hi_all <= lo_all
 };
 
-__device__ __forceinline__ Ranges key_tile_ranges(const Params& p, int q_row0) {
-  Ranges R;
+// The r-th item of this CTA (snake over cost-ordered items), or -1.
+__device__ __forceinline__ int item_index(const Params& p, int r) {
+  const int P = gridDim.x, c = blockIdx.x;
+  const int k = r * P + ((r & 1) ? (P - 1 - c) : c);
+  return k < p.n_items ? k : -1;
+}
+
+__device__ __forceinline__ Item make_item(const Params& p, int k) {
+  Item it;
+  const int BH = p.B * p.Hq;
+  it.bh = k % BH;
+  const int qb = p.n_qblocks - 1 - k / BH;   // costliest (latest) query blocks first
+  it.b = it.bh / p.Hq;
+  it.g = (it.bh % p.Hq) / (p.Hq / p.Hkv);
+  it.q_row0 = qb * (NQ * BM);
   const int off = p.Skv - p.Sq;
   const int n_kt = (p.Skv + BN - 1) / BN;
-  R.lo_all = 1 << 30;
-  R.hi_all = 0;
+  it.lo_all = 1 << 30;
+  it.hi_all = 0;
 #pragma unroll
   for (int i = 0; i < NQ; ++i) {
-    const int r0 = q_row0 + BM * i;
+    const int r0 = it.q_row0 + BM * i;
     const int r1 = min(r0 + BM, p.Sq);   // exclusive
     int lo = 0, hi = 0;
     if (r0 < p.Sq) {
       if (!p.causal) {
-        lo = 0;
         hi = n_kt;
       } else {
         const int last_key = min(r1 - 1 + off, p.Skv - 1);
@@ -96,18 +122,20 @@ __device__ __forceinline__ Ranges key_tile_ranges(const Params& p, int q_row0) {
         }
       }
     }
-    R.lo[i] = lo;
-    R.hi[i] = hi;
+    it.lo[i] = lo;
+    it.hi[i] = hi;
     if (hi > lo) {
-      R.lo_all = min(R.lo_all, lo);
-      R.hi_all = max(R.hi_all, hi);
+      it.lo_all = min(it.lo_all, lo);
+      it.hi_all = max(it.hi_all, hi);
     }
   }
-  if (R.hi_all <= 0) R.lo_all = R.hi_all = 0;
-  return R;
+  if (it.hi_all <= 0) it.lo_all = it.hi_all = 0;
+  return it;
 }
 
-// True if every (row, key) pair of query tile rows [r0, r0+BM) x key tile j is visible.
+__device__ __forceinline__ bool active(const Item& it, int i, int j) { return j >= it.lo[i] && j < it.hi[i]; }
+
+// True if every (row, key) pair of query rows [r0, r0+BM) x key tile j is visible.
 __device__ __forceinline__ bool tile_unmasked(const Params& p, int r0, int j) {
   const int off = p.Skv - p.Sq;
   const int k0 = j * BN, k1 = j * BN + BN - 1;
@@ -123,15 +151,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_v, const Params p) {
   using C = Cfg<D>;
-  constexpr int STAGES = C::STAGES;
+  constexpr int STAGES = C::STAGES, QBUF = C::QBUF;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sQ = smem;                                   // [NQ][KATOMS][BM rows x 128 B]
-  uint8_t* sRing = smem + NQ * C::Q_BYTES;              // [STAGES][KATOMS][BN rows x 128 B]
+  uint8_t* sQ = smem;                                   // [QBUF][NQ][KATOMS][BM rows x 128 B]
+  uint8_t* sRing = smem + QBUF * NQ * C::Q_BYTES;       // [STAGES][KATOMS][BN rows x 128 B]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sRing + STAGES * C::TILE_BYTES);
-  uint64_t* q_full = bars;                              // 1
-  uint64_t* full = bars + 1;                            // STAGES
+  uint64_t* q_full = bars;                              // QBUF
+  uint64_t* q_empty = q_full + QBUF;                    // QBUF
+  uint64_t* full = q_empty + QBUF;                      // STAGES
   uint64_t* empty = full + STAGES;                      // STAGES
   uint64_t* s_ready = empty + STAGES;                   // NQ
   uint64_t* p_ready = s_ready + NQ;                     // NQ
@@ -141,18 +170,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  // heaviest query blocks first: block-major over (b, h) for the last query block, ...
-  const int BH = p.B * p.Hq;
-  const int bh = blockIdx.x % BH;
-  const int qb = p.n_qblocks - 1 - static_cast<int>(blockIdx.x / BH);
-  const int b = bh / p.Hq, h = bh % p.Hq;
-  const int g = h / (p.Hq / p.Hkv);
-  const int q_row0 = qb * (NQ * BM);
-  const Ranges R = key_tile_ranges(p, q_row0);
+  const int n_rounds = (p.n_items + gridDim.x - 1) / gridDim.x;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    for (int q = 0; q < QBUF; ++q) {
+      mbar_init(&q_full[q], 1);
+      mbar_init(&q_empty[q], 1);
+    }
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -175,207 +199,260 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == kTmaWarp) {
+  if (warp >= 8) {
+   // ------------------------------------------------------------ producer warpgroup
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
+   if (warp == kTmaWarp) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && R.hi_all > R.lo_all) {
+    if (lane == 0) {
       prefetch_tmap(&tmap_q);
       prefetch_tmap(&tmap_k);
       prefetch_tmap(&tmap_v);
-      mbar_arrive_expect_tx(q_full, NQ * C::Q_BYTES);
-      for (int i = 0; i < NQ; ++i)
-        for (int a = 0; a < C::KATOMS; ++a)
-          tma_load_3d(sQ + (i * C::KATOMS + a) * BM * 128, &tmap_q, q_full, a * 64, q_row0 + BM * i, bh);
-      const int kv_plane = b * p.Hkv + g;
-      int n = 0;
+      int n = 0, qn = 0;
       bool ok = true;
-      for (int j = R.lo_all; j < R.hi_all && ok; ++j) {
-        for (int kv = 0; kv < 2 && ok; ++kv, ++n) {
-          const int st = n % STAGES;
-          if (!mbar_wait(&empty[st], ((n / STAGES) & 1) ^ 1, abort_flag, p.err)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&full[st], C::TILE_BYTES);
-          const CUtensorMap* tm = kv ? &tmap_v : &tmap_k;
+      for (int r = 0; r < n_rounds && ok; ++r) {
+        const int k = item_index(p, r);
+        if (k < 0) continue;
+        const Item it = make_item(p, k);
+        if (it.hi_all <= it.lo_all) continue;
+        const int qb = qn % QBUF;
+        if (qn >= QBUF && !(ok = mbar_wait(&q_empty[qb], ((qn / QBUF) - 1) & 1, abort_flag, p.err))) break;
+        mbar_arrive_expect_tx(&q_full[qb], NQ * C::Q_BYTES);
+        for (int i = 0; i < NQ; ++i)
           for (int a = 0; a < C::KATOMS; ++a)
-            tma_load_3d(sRing + st * C::TILE_BYTES + a * BN * 128, tm, &full[st], a * 64, j * BN, kv_plane);
+            tma_load_3d(sQ + ((qb * NQ + i) * C::KATOMS + a) * BM * 128, &tmap_q, &q_full[qb], a * 64,
+                        it.q_row0 + BM * i, it.bh);
+        ++qn;
+        const int kv_plane = it.b * p.Hkv + it.g;
+        for (int j = it.lo_all; j < it.hi_all && ok; ++j) {
+          for (int kv = 0; kv < 2; ++kv, ++n) {
+            const int st = n % STAGES;
+            if (!(ok = mbar_wait(&empty[st], ((n / STAGES) & 1) ^ 1, abort_flag, p.err))) break;
+            mbar_arrive_expect_tx(&full[st], C::TILE_BYTES);
+            const CUtensorMap* tm = kv ? &tmap_v : &tmap_k;
+            for (int a = 0; a < C::KATOMS; ++a)
+              tma_load_3d(sRing + st * C::TILE_BYTES + a * BN * 128, tm, &full[st], a * 64, j * BN, kv_plane);
+          }
         }
       }
       // the last loads issued must land before the CTA may exit (normally already consumed)
       for (int k = max(0, n - STAGES); k < n; ++k) mbar_wait(&full[k % STAGES], (k / STAGES) & 1, nullptr, p.err);
     }
-  } else if (warp == kMmaWarp) {
+   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && R.hi_all > R.lo_all) {
+    if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(BM, BN, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, 0, 1);
-      const uint32_t q_addr = smem_u32(sQ);
+      const uint32_t q_base = smem_u32(sQ);
       const uint32_t ring_addr = smem_u32(sRing);
-      int n = 0;
-      int t[NQ] = {0, 0};
-      bool ok = mbar_wait(q_full, 0, abort_flag, p.err);
-      tc_fence_after();
-      for (int j = R.lo_all; j < R.hi_all && ok; ++j) {
-        // ---- S_i = Q_i K_j^T
-        int st = n % STAGES;
-        if (!(ok = mbar_wait(&full[st], (n / STAGES) & 1, abort_flag, p.err))) break;
-        tc_fence_after();
+      int n = 0, qn = 0;
+      int ts[NQ] = {0, 0};
+      bool ok = true;
+
+      auto issue_s = [&](int i, int qb, int st) {  // S_i = Q_i K^T from ring slot st
+        const uint32_t d_tmem = tmem + C::S_COL + 128 * i;
+        const uint32_t q_addr = q_base + (qb * NQ + i) * C::Q_BYTES;
 #pragma unroll
-        for (int i = 0; i < NQ; ++i) {
-          if (j < R.lo[i] || j >= R.hi[i]) continue;
-          const uint32_t d_tmem = tmem + C::S_COL + 128 * i;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t koff = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-            const uint64_t adesc = sw128_desc(q_addr + i * C::Q_BYTES + koff, 16, 1024);
-            const uint64_t bdesc = sw128_desc(ring_addr + st * C::TILE_BYTES + koff, 16, 1024);
-            mma_ss(d_tmem, adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(&s_ready[i]);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+          mma_ss(d_tmem, sw128_desc(q_addr + koff, 16, 1024),
+                 sw128_desc(ring_addr + st * C::TILE_BYTES + koff, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&empty[st]);
-        ++n;
-        // ---- O_i += P_i V_j
+        mma_commit(&s_ready[i]);
+      };
+      auto wait_slot = [&](int& st) -> bool {   // next ring slot, in load order
         st = n % STAGES;
-        if (!(ok = mbar_wait(&full[st], (n / STAGES) & 1, abort_flag, p.err))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int i = 0; i < NQ; ++i) {
-          if (j < R.lo[i] || j >= R.hi[i]) continue;
-          if (!(ok = mbar_wait(&p_ready[i], t[i] & 1, abort_flag, p.err))) break;
-          tc_fence_after();
-          const uint32_t o_tmem = tmem + C::O_COL + D * i;
-          const uint32_t p_tmem = tmem + C::S_COL + 128 * i;
-#pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint64_t bdesc = sw128_desc(ring_addr + st * C::TILE_BYTES + kk * 16 * 128, BN * 128, 1024);
-            mma_ts(o_tmem, p_tmem + kk * 8, bdesc, idesc_pv, (j > R.lo[i] || kk > 0) ? 1u : 0u);
-          }
-          ++t[i];
-        }
-        if (!ok) break;
-        mma_commit(&empty[st]);
+        const bool r = mbar_wait(&full[st], (n / STAGES) & 1, abort_flag, p.err);
         ++n;
+        tc_fence_after();
+        return r;
+      };
+
+      for (int r = 0; r < n_rounds && ok; ++r) {
+        const int k = item_index(p, r);
+        if (k < 0) continue;
+        const Item it = make_item(p, k);
+        if (it.hi_all <= it.lo_all) continue;
+        const int qb = qn % QBUF;
+        if (!(ok = mbar_wait(&q_full[qb], (qn / QBUF) & 1, abort_flag, p.err))) break;
+        tc_fence_after();
+        ++qn;
+        // prologue: S_i(lo) for the tiles that start at the first key tile
+        int stK;
+        if (!(ok = wait_slot(stK))) break;
 #pragma unroll
         for (int i = 0; i < NQ; ++i)
-          if (j == R.hi[i] - 1) mma_commit(&o_done[i]);
+          if (active(it, i, it.lo_all)) issue_s(i, qb, stK);
+        mma_commit(&empty[stK]);
+        if (it.hi_all - it.lo_all == 1) mma_commit(&q_empty[qb]);
+
+        for (int j = it.lo_all; j < it.hi_all && ok; ++j) {
+          int stV;
+          if (!(ok = wait_slot(stV))) break;
+          const bool next = j + 1 < it.hi_all;
+          int stK1 = -1;
+#pragma unroll
+          for (int i = 0; i < NQ; ++i) {
+            if (active(it, i, j)) {
+              if (!(ok = mbar_wait(&p_ready[i], ts[i] & 1, abort_flag, p.err))) break;
+              tc_fence_after();
+              ++ts[i];
+              const uint32_t o_tmem = tmem + C::O_COL + D * i;
+              const uint32_t p_tmem = tmem + C::S_COL + 128 * i;
+#pragma unroll
+              for (int kk = 0; kk < BN / 16; ++kk)
+                mma_ts(o_tmem, p_tmem + kk * 8,
+                       sw128_desc(ring_addr + stV * C::TILE_BYTES + kk * 16 * 128, BN * 128, 1024), idesc_pv,
+                       (j > it.lo[i] || kk > 0) ? 1u : 0u);
+              if (j == it.hi[i] - 1) mma_commit(&o_done[i]);
+            }
+            if (next && active(it, i, j + 1)) {
+              if (stK1 < 0 && !(ok = wait_slot(stK1))) break;
+              issue_s(i, qb, stK1);
+            }
+          }
+          if (!ok) break;
+          if (next && stK1 < 0 && !(ok = wait_slot(stK1))) break;   // K tile that no query tile needs
+          mma_commit(&empty[stV]);
+          if (next) mma_commit(&empty[stK1]);
+          if (j == it.hi_all - 2) mma_commit(&q_empty[qb]);
+        }
       }
       // everything issued above must be complete before tensor memory is released
       mma_commit(drain);
       mbar_wait(drain, 0, nullptr, p.err);
     }
+   }
   } else {
     // ------------------------------------------------------------ softmax groups
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
     const int i = warp >> 2;                 // query tile
     const int wq = warp & 3;                 // lane quarter of tensor memory
     const int rl = wq * 32 + lane;           // row within the tile
-    const int r = q_row0 + BM * i + rl;      // query row
     const int off = p.Skv - p.Sq;
     const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t s_tmem = tmem + lane_bits + C::S_COL + 128 * i;
     const uint32_t o_tmem = tmem + lane_bits + C::O_COL + D * i;
-    // visible keys of this row: [key_lo, key_hi]
-    const int key_hi = p.causal ? min(r + off, p.Skv - 1) : p.Skv - 1;
-    const int key_lo = (p.causal && p.window > 0) ? r + off - p.window + 1 : 0;
-    const int my_lo = (i == 0) ? R.lo[0] : R.lo[1];
-    const int my_hi = (i == 0) ? R.hi[0] : R.hi[1];
-    const bool have_keys = my_hi > my_lo;
-
-    float m_ref = -INFINITY, l = 0.f;
+    const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
+    int t = 0, oc = 0;
     bool ok = true;
-    for (int j = my_lo, t = 0; j < my_hi; ++j, ++t) {
-      ok = mbar_wait(&s_ready[i], t & 1, abort_flag, p.err);
+
+    for (int rr = 0; rr < n_rounds && ok; ++rr) {
+      const int k = item_index(p, rr);
+      if (k < 0) continue;
+      const Item it = make_item(p, k);
+      const int my_lo = (i == 0) ? it.lo[0] : it.lo[1];
+      const int my_hi = (i == 0) ? it.hi[0] : it.hi[1];
+      const int r0 = it.q_row0 + BM * i;
+      const int r = r0 + rl;                 // query row of this thread
+      const bool store = r < p.Sq;
+      __nv_bfloat16* orow = p.out + (static_cast<size_t>(it.bh) * p.Sq + r) * D;
+      if (my_hi <= my_lo) {                  // no visible key for any row of this tile
+        if (store) {
+          uint4* dst = reinterpret_cast<uint4*>(orow);
+          for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        continue;
+      }
+      // visible keys of this row: [key_lo, key_hi]
+      const int key_hi = p.causal ? min(r + off, p.Skv - 1) : p.Skv - 1;
+      const int key_lo = (p.causal && p.window > 0) ? r + off - p.window + 1 : 0;
+      float m_ref = -INFINITY, l = 0.f;
+
+      for (int j = my_lo; j < my_hi; ++j, ++t) {
+        ok = mbar_wait(&s_ready[i], t & 1, abort_flag, p.err);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float s[BN];
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) tmem_ld32f(s_tmem + 32 * c, s + 32 * c);
+        tmem_wait_ld();
+        if (!tile_unmasked(p, r0, j)) {
+          const int c_lo = key_lo - j * BN, c_hi = key_hi - j * BN;
+#pragma unroll
+          for (int c = 0; c < BN; ++c) s[c] = (c >= c_lo && c <= c_hi) ? s[c] : -INFINITY;
+        }
+        float mx = fmax3(s[0], s[1], s[2]);
+#pragma unroll
+        for (int c = 3; c < BN - 1; c += 2) mx = fmax3(mx, s[c], s[c + 1]);
+        mx = fmaxf(mx, s[BN - 1]);
+        const float m_tile = mx * p.scale_log2;
+        float alpha = 1.f;
+        if (m_tile > m_ref + kTau) {
+          alpha = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - m_tile);
+          l *= alpha;
+          m_ref = m_tile;
+        }
+        const bool rescale = (j > my_lo) && (alpha != 1.f);
+        if (__any_sync(0xffffffffu, rescale)) {
+          const uint64_t a2 = f2_pack(alpha, alpha);
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(o_tmem + 32 * c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              float x0, x1;
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2), x0, x1);
+              o[e] = __float_as_uint(x0);
+              o[e + 1] = __float_as_uint(x1);
+            }
+            tmem_st32(o_tmem + 32 * c, o);
+          }
+        }
+        const float mb = (m_ref == -INFINITY) ? 0.f : m_ref;
+        const uint64_t nm2 = f2_pack(-mb, -mb);
+        uint32_t pk[BN / 2];
+        uint64_t sum2 = f2_pack(0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < BN; c += 2) {
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), c2, nm2), x0, x1);
+          const float p0 = ex2(x0), p1 = ex2(x1);
+          sum2 = f2_add(sum2, f2_pack(p0, p1));
+          pk[c / 2] = pack_bf16x2(p0, p1);
+        }
+        float s0, s1;
+        f2_unpack(sum2, s0, s1);
+        l += s0 + s1;
+#pragma unroll
+        for (int c = 0; c < BN / 64; ++c) tmem_st32(s_tmem + 32 * c, pk + 32 * c);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_ready[i]);
+      }
+      if (!ok) break;
+      // ---- epilogue: O / l -> bf16 (tcgen05.ld is warp-collective: every lane loads)
+      ok = mbar_wait(&o_done[i], oc & 1, abort_flag, p.err);
+      ++oc;
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t sr[BN];
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) tmem_ld32(s_tmem + 32 * c, sr + 32 * c);
-      tmem_wait_ld();
-      float s[BN];
-#pragma unroll
-      for (int c = 0; c < BN; ++c) s[c] = __uint_as_float(sr[c]);
-      if (!tile_unmasked(p, q_row0 + BM * i, j)) {
-        const int c_lo = key_lo - j * BN, c_hi = key_hi - j * BN;
-#pragma unroll
-        for (int c = 0; c < BN; ++c) s[c] = (c >= c_lo && c <= c_hi) ? s[c] : -INFINITY;
-      }
-      float mx = s[0];
-#pragma unroll
-      for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
-      const float m_tile = mx * p.scale_log2;
-      float alpha = 1.f;
-      if (m_tile > m_ref + kTau) {
-        alpha = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - m_tile);
-        l *= alpha;
-        m_ref = m_tile;
-      }
-      const bool rescale = (t > 0) && (alpha != 1.f);
-      if (__any_sync(0xffffffffu, rescale)) {
+      const float inv = (l > 0.f) ? 1.f / l : 0.f;
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(o_tmem + 32 * c, o);
-          tmem_wait_ld();
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(o_tmem + 32 * c, o);
+        tmem_wait_ld();
+        uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(o_tmem + 32 * c, o);
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+        if (store) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
         }
       }
-      const float mb = (m_ref == -INFINITY) ? 0.f : m_ref;
-      uint32_t pk[BN / 2];
-      float lsum = 0.f;
-#pragma unroll
-      for (int c = 0; c < BN; c += 2) {
-        const float p0 = ex2(fmaf(s[c], p.scale_log2, -mb));
-        const float p1 = ex2(fmaf(s[c + 1], p.scale_log2, -mb));
-        lsum += p0 + p1;
-        pk[c / 2] = pack_bf16x2(p0, p1);
-      }
-      l += lsum;
-#pragma unroll
-      for (int c = 0; c < BN / 64; ++c)
-        tmem_st32(s_tmem + 32 * c, pk + 32 * c);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&p_ready[i]);
+      tc_fence_before();   // this group's O reads precede the next item's first P_i V product
     }
-    // ---- epilogue: O / l -> bf16
-    if (ok && have_keys) {
-      ok = mbar_wait(&o_done[i], 0, abort_flag, p.err);
-      ok = __all_sync(0xffffffffu, ok);
-    }
-    // tcgen05.ld is warp-collective (.sync.aligned): every lane loads, only rows < Sq store
-    if (ok) {
-      __nv_bfloat16* orow = p.out + (static_cast<size_t>(bh) * p.Sq + r) * D;
-      const bool store = r < p.Sq;
-      if (have_keys) {
-        tc_fence_after();
-        const float inv = (l > 0.f) ? 1.f / l : 0.f;
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(o_tmem + 32 * c, o);
-          tmem_wait_ld();
-          uint4 pk4[4];
-          uint32_t* pk = reinterpret_cast<uint32_t*>(pk4);
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
-          if (store) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) dst[e] = pk4[e];
-          }
-        }
-      } else if (store) {
-        uint4* dst = reinterpret_cast<uint4*>(orow);
-        for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
-      }
-    }
-    // if a wait gave up, the rows stay unwritten and the error word records it
+    // if a wait gave up, the remaining rows stay unwritten and the error word records it
   }
 
   tc_fence_before();
@@ -418,6 +495,19 @@ bool make_map(CUtensorMap* m, const void* base, int D, int rows, int planes) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+int sm_count() {
+  constexpr int kMaxDevices = 64;
+  static int cache[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
 template <int D>
 cudaError_t launch_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const Params& p,
                      cudaStream_t stream) {
@@ -425,7 +515,15 @@ cudaError_t launch_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   const size_t smem = Cfg<D>::SMEM;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const unsigned grid = static_cast<unsigned>(p.n_qblocks) * static_cast<unsigned>(p.B * p.Hq);
+  // setmaxnreg.inc waits until the block's own registers can cover the request:
+  // refuse to launch a build whose allocation could not.
+  cudaFuncAttributes fa{};
+  e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs * kThreads < 128 * (2 * kSoftmaxRegs + kProducerRegs)) return cudaErrorInvalidConfiguration;
+  const int sms = sm_count();
+  if (sms <= 0) return cudaErrorInvalidDevice;
+  const unsigned grid = static_cast<unsigned>(min(p.n_items, sms));
   kern<<<grid, kThreads, smem, stream>>>(mq, mk, mv, p);
   return cudaGetLastError();
 }
@@ -447,6 +545,9 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, void*
   p.causal = causal;
   p.window = window;
   p.n_qblocks = (Sq + NQ * BM - 1) / (NQ * BM);
+  const long long items = static_cast<long long>(p.n_qblocks) * B * Hq;
+  if (items > (1LL << 30)) return cudaErrorInvalidValue;
+  p.n_items = static_cast<int>(items);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.err = err;
