@@ -60,6 +60,12 @@ constexpr int kSoftmaxRegs = 200;
 constexpr int kProducerRegs = 104;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kTau = 8.0f;     // lazy-rescale threshold, log2 units
+// Of every 16 score pairs of a row, how many take exp2 on the FMA pipe
+// (exp2_fma2) instead of the MUFU unit, which is the bottleneck of the softmax.
+#ifndef ATTN_EXP_EMU
+#define ATTN_EXP_EMU 0
+#endif
+constexpr int kEmuPer16 = ATTN_EXP_EMU;
 
 template <int D>
 struct Cfg {
@@ -68,8 +74,16 @@ struct Cfg {
   static constexpr int Q_BYTES = BM * D * 2;          // one query tile
   static constexpr int QBUF = (D == 128) ? 1 : 2;     // query buffers (items in flight)
   static constexpr int STAGES = (D == 128) ? 4 : 6;   // ring slots; K and V tiles alternate
+  // D = 64 leaves room in tensor memory for P buffers of their own (SEP_P):
+  // S_i [128 i, +128), P_i [256 + 64 i, +64), O_i [384 + 64 i, +64).  The
+  // softmax then releases S_i as soon as it has loaded it, and S_i(j+1) is
+  // computed while the softmax of tile j is still running.  D = 128 has no
+  // room: P_i is written over the first 64 columns of S_i, O_i [256 + 128 i, +128).
+  static constexpr bool SEP_P = (D == 64);
   static constexpr uint32_t S_COL = 0;                // + 128 * i
-  static constexpr uint32_t O_COL = 256;              // + D * i
+  static constexpr uint32_t P_COL = SEP_P ? 256 : 0;  // + (SEP_P ? 64 : 128) * i
+  static constexpr uint32_t P_STRIDE = SEP_P ? 64 : 128;
+  static constexpr uint32_t O_COL = SEP_P ? 384 : 256;  // + D * i
   static constexpr size_t SMEM = 1024 /*align*/ + QBUF * NQ * Q_BYTES + STAGES * TILE_BYTES + 256;
 };
 
@@ -164,8 +178,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = full + STAGES;                      // STAGES
   uint64_t* s_ready = empty + STAGES;                   // NQ
   uint64_t* p_ready = s_ready + NQ;                     // NQ
-  uint64_t* o_done = p_ready + NQ;                      // NQ
-  uint64_t* drain = o_done + NQ;                        // 1
+  uint64_t* o_done = p_ready + NQ;                      // NQ: O_i final (SEP_P: each P_i V done)
+  uint64_t* s_free = o_done + NQ;                       // NQ: S_i loaded by the softmax (SEP_P)
+  uint64_t* drain = s_free + NQ;                        // 1
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -185,6 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s_ready[i], 1);
       mbar_init(&p_ready[i], 4 * 32);
       mbar_init(&o_done[i], 1);
+      mbar_init(&s_free[i], 4 * 32);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -224,14 +240,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                         it.q_row0 + BM * i, it.bh);
         ++qn;
         const int kv_plane = it.b * p.Hkv + it.g;
-        for (int j = it.lo_all; j < it.hi_all && ok; ++j) {
-          for (int kv = 0; kv < 2; ++kv, ++n) {
-            const int st = n % STAGES;
-            if (!(ok = mbar_wait(&empty[st], ((n / STAGES) & 1) ^ 1, abort_flag, p.err))) break;
-            mbar_arrive_expect_tx(&full[st], C::TILE_BYTES);
-            const CUtensorMap* tm = kv ? &tmap_v : &tmap_k;
-            for (int a = 0; a < C::KATOMS; ++a)
-              tma_load_3d(sRing + st * C::TILE_BYTES + a * BN * 128, tm, &full[st], a * 64, j * BN, kv_plane);
+        auto load = [&](bool is_v, int j) -> bool {   // next ring slot <- K_j or V_j
+          const int st = n % STAGES;
+          if (!mbar_wait(&empty[st], ((n / STAGES) & 1) ^ 1, abort_flag, p.err)) return false;
+          mbar_arrive_expect_tx(&full[st], C::TILE_BYTES);
+          const CUtensorMap* tm = is_v ? &tmap_v : &tmap_k;
+          for (int a = 0; a < C::KATOMS; ++a)
+            tma_load_3d(sRing + st * C::TILE_BYTES + a * BN * 128, tm, &full[st], a * 64, j * BN, kv_plane);
+          ++n;
+          return true;
+        };
+        // load order = the MMA thread's consumption order
+        if constexpr (C::SEP_P) {   // K_lo, then K_{j+1} ahead of V_j
+          ok = load(false, it.lo_all);
+          for (int j = it.lo_all; j < it.hi_all && ok; ++j) {
+            if (j + 1 < it.hi_all) ok = load(false, j + 1);
+            if (ok) ok = load(true, j);
+          }
+        } else {                    // K_j, V_j
+          for (int j = it.lo_all; j < it.hi_all && ok; ++j) {
+            ok = load(false, j);
+            if (ok) ok = load(true, j);
           }
         }
       }
@@ -243,20 +272,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(BM, BN, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, 0, 1);
-      const uint32_t q_base = smem_u32(sQ);
-      const uint32_t ring_addr = smem_u32(sRing);
+      constexpr uint32_t kHi = sw128_desc_hi(1024);   // 8-row groups 1024 B apart
+      // descriptor low words at K step 0: Q tiles (K-major), ring slots as K (K-major)
+      // and as V (MN-major, 64-column blocks BN*128 bytes apart); a K step adds a
+      // compile-time offset in 16-byte units
+      const uint32_t q_lo0 = sw128_desc_lo(smem_u32(sQ), 16);
+      const uint32_t k_lo0 = sw128_desc_lo(smem_u32(sRing), 16);
+      const uint32_t v_lo0 = sw128_desc_lo(smem_u32(sRing), BN * 128);
       int n = 0, qn = 0;
       int ts[NQ] = {0, 0};
       bool ok = true;
 
       auto issue_s = [&](int i, int qb, int st) {  // S_i = Q_i K^T from ring slot st
         const uint32_t d_tmem = tmem + C::S_COL + 128 * i;
-        const uint32_t q_addr = q_base + (qb * NQ + i) * C::Q_BYTES;
+        const uint32_t a_lo = q_lo0 + (((qb * NQ + i) * C::Q_BYTES) >> 4);
+        const uint32_t b_lo = k_lo0 + ((st * C::TILE_BYTES) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-          mma_ss(d_tmem, sw128_desc(q_addr + koff, 16, 1024),
-                 sw128_desc(ring_addr + st * C::TILE_BYTES + koff, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+          const uint32_t koff = ((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4;
+          mma_ss(d_tmem, desc64(a_lo + koff, kHi), desc64(b_lo + koff, kHi), idesc_s, kk > 0 ? 1u : 0u);
         }
         mma_commit(&s_ready[i]);
       };
@@ -268,54 +302,126 @@ __global__ void __launch_bounds__(kThreads, 1)
         return r;
       };
 
-      for (int r = 0; r < n_rounds && ok; ++r) {
-        const int k = item_index(p, r);
-        if (k < 0) continue;
-        const Item it = make_item(p, k);
-        if (it.hi_all <= it.lo_all) continue;
-        const int qb = qn % QBUF;
-        if (!(ok = mbar_wait(&q_full[qb], (qn / QBUF) & 1, abort_flag, p.err))) break;
-        tc_fence_after();
-        ++qn;
-        // prologue: S_i(lo) for the tiles that start at the first key tile
-        int stK;
-        if (!(ok = wait_slot(stK))) break;
+      if constexpr (C::SEP_P) {
+        // Order per key tile j: S_i(j+1) as soon as softmax group i has loaded
+        // S_i(j) (s_free), then P_i(j) V_j as soon as it has written P_i(j).
+        int tf[NQ] = {0, 0};    // s_free phases consumed per tile
+        for (int r = 0; r < n_rounds && ok; ++r) {
+          const int k = item_index(p, r);
+          if (k < 0) continue;
+          const Item it = make_item(p, k);
+          if (it.hi_all <= it.lo_all) continue;
+          const int qb = qn % QBUF;
+          if (!(ok = mbar_wait(&q_full[qb], (qn / QBUF) & 1, abort_flag, p.err))) break;
+          tc_fence_after();
+          ++qn;
+          int stK;
+          if (!(ok = wait_slot(stK))) break;
 #pragma unroll
-        for (int i = 0; i < NQ; ++i)
-          if (active(it, i, it.lo_all)) issue_s(i, qb, stK);
-        mma_commit(&empty[stK]);
-        if (it.hi_all - it.lo_all == 1) mma_commit(&q_empty[qb]);
+          for (int i = 0; i < NQ; ++i)
+            if (active(it, i, it.lo_all)) issue_s(i, qb, stK);
+          mma_commit(&empty[stK]);
+          if (it.hi_all - it.lo_all == 1) mma_commit(&q_empty[qb]);
 
-        for (int j = it.lo_all; j < it.hi_all && ok; ++j) {
-          int stV;
-          if (!(ok = wait_slot(stV))) break;
-          const bool next = j + 1 < it.hi_all;
-          int stK1 = -1;
+          for (int j = it.lo_all; j < it.hi_all && ok; ++j) {
+            if (j + 1 < it.hi_all) {
+              int stK1;
+              if (!(ok = wait_slot(stK1))) break;
 #pragma unroll
-          for (int i = 0; i < NQ; ++i) {
-            if (active(it, i, j)) {
+              for (int i = 0; i < NQ; ++i) {
+                if (!active(it, i, j + 1)) continue;
+                if (active(it, i, j)) {   // S_i still holds tile j until the softmax has loaded it
+                  if (!(ok = mbar_wait(&s_free[i], tf[i] & 1, abort_flag, p.err))) break;
+                  tc_fence_after();
+                  ++tf[i];
+                }
+                issue_s(i, qb, stK1);
+              }
+              if (!ok) break;
+              mma_commit(&empty[stK1]);
+              if (j + 1 == it.hi_all - 1) mma_commit(&q_empty[qb]);
+            }
+            int stV;
+            if (!(ok = wait_slot(stV))) break;
+#pragma unroll
+            for (int i = 0; i < NQ; ++i) {
+              if (!active(it, i, j)) continue;
               if (!(ok = mbar_wait(&p_ready[i], ts[i] & 1, abort_flag, p.err))) break;
               tc_fence_after();
               ++ts[i];
               const uint32_t o_tmem = tmem + C::O_COL + D * i;
-              const uint32_t p_tmem = tmem + C::S_COL + 128 * i;
+              const uint32_t p_tmem = tmem + C::P_COL + C::P_STRIDE * i;
+              const uint32_t vb_lo = v_lo0 + ((stV * C::TILE_BYTES) >> 4);
+              const uint32_t acc0 = (j > it.lo[i]) ? 1u : 0u;
 #pragma unroll
               for (int kk = 0; kk < BN / 16; ++kk)
-                mma_ts(o_tmem, p_tmem + kk * 8,
-                       sw128_desc(ring_addr + stV * C::TILE_BYTES + kk * 16 * 128, BN * 128, 1024), idesc_pv,
-                       (j > it.lo[i] || kk > 0) ? 1u : 0u);
-              if (j == it.hi[i] - 1) mma_commit(&o_done[i]);
+                mma_ts(o_tmem, p_tmem + kk * 8, desc64(vb_lo + ((kk * 16 * 128) >> 4), kHi), idesc_pv,
+                       kk > 0 ? 1u : acc0);
+              mma_commit(&o_done[i]);   // P_i free again, O_i current
             }
-            if (next && active(it, i, j + 1)) {
-              if (stK1 < 0 && !(ok = wait_slot(stK1))) break;
-              issue_s(i, qb, stK1);
+            if (!ok) break;
+            mma_commit(&empty[stV]);
+          }
+          // tiles whose last S tile was loaded but never freed by a following S: consume the phase
+#pragma unroll
+          for (int i = 0; i < NQ; ++i) {
+            if (it.hi[i] > it.lo[i] && ok) {
+              if (!(ok = mbar_wait(&s_free[i], tf[i] & 1, abort_flag, p.err))) break;
+              ++tf[i];
             }
           }
-          if (!ok) break;
-          if (next && stK1 < 0 && !(ok = wait_slot(stK1))) break;   // K tile that no query tile needs
-          mma_commit(&empty[stV]);
-          if (next) mma_commit(&empty[stK1]);
-          if (j == it.hi_all - 2) mma_commit(&q_empty[qb]);
+        }
+      } else {
+      for (int r = 0; r < n_rounds && ok; ++r) {
+          const int k = item_index(p, r);
+          if (k < 0) continue;
+          const Item it = make_item(p, k);
+          if (it.hi_all <= it.lo_all) continue;
+          const int qb = qn % QBUF;
+          if (!(ok = mbar_wait(&q_full[qb], (qn / QBUF) & 1, abort_flag, p.err))) break;
+          tc_fence_after();
+          ++qn;
+          // prologue: S_i(lo) for the tiles that start at the first key tile
+          int stK;
+          if (!(ok = wait_slot(stK))) break;
+#pragma unroll
+          for (int i = 0; i < NQ; ++i)
+            if (active(it, i, it.lo_all)) issue_s(i, qb, stK);
+          mma_commit(&empty[stK]);
+          if (it.hi_all - it.lo_all == 1) mma_commit(&q_empty[qb]);
+
+          for (int j = it.lo_all; j < it.hi_all && ok; ++j) {
+            int stV;
+            if (!(ok = wait_slot(stV))) break;
+            const bool next = j + 1 < it.hi_all;
+            int stK1 = -1;
+#pragma unroll
+            for (int i = 0; i < NQ; ++i) {
+              if (active(it, i, j)) {
+                if (!(ok = mbar_wait(&p_ready[i], ts[i] & 1, abort_flag, p.err))) break;
+                tc_fence_after();
+                ++ts[i];
+                const uint32_t o_tmem = tmem + C::O_COL + D * i;
+                const uint32_t p_tmem = tmem + C::P_COL + C::P_STRIDE * i;
+                const uint32_t vb_lo = v_lo0 + ((stV * C::TILE_BYTES) >> 4);
+                const uint32_t acc0 = (j > it.lo[i]) ? 1u : 0u;
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk)
+                  mma_ts(o_tmem, p_tmem + kk * 8, desc64(vb_lo + ((kk * 16 * 128) >> 4), kHi), idesc_pv,
+                         kk > 0 ? 1u : acc0);
+                if (j == it.hi[i] - 1) mma_commit(&o_done[i]);
+              }
+              if (next && active(it, i, j + 1)) {
+                if (stK1 < 0 && !(ok = wait_slot(stK1))) break;
+                issue_s(i, qb, stK1);
+              }
+            }
+            if (!ok) break;
+            if (next && stK1 < 0 && !(ok = wait_slot(stK1))) break;   // K tile that no query tile needs
+            mma_commit(&empty[stV]);
+            if (next) mma_commit(&empty[stK1]);
+            if (j == it.hi_all - 2) mma_commit(&q_empty[qb]);
+          }
         }
       }
       // everything issued above must be complete before tensor memory is released
@@ -332,9 +438,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int off = p.Skv - p.Sq;
     const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t s_tmem = tmem + lane_bits + C::S_COL + 128 * i;
+    const uint32_t p_tmem = tmem + lane_bits + C::P_COL + C::P_STRIDE * i;
     const uint32_t o_tmem = tmem + lane_bits + C::O_COL + D * i;
     const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
     int t = 0, oc = 0;
+    int pv = 0;   // SEP_P: P_i V products of this tile completed and waited for
     bool ok = true;
 
     for (int rr = 0; rr < n_rounds && ok; ++rr) {
@@ -370,21 +478,40 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < BN / 32; ++c) tmem_ld32f(s_tmem + 32 * c, s + 32 * c);
         tmem_wait_ld();
+        if constexpr (C::SEP_P) {   // S_i may be overwritten by S_i(j+1) from here on
+          tc_fence_before();
+          mbar_arrive(&s_free[i]);
+        }
         if (!tile_unmasked(p, r0, j)) {
           const int c_lo = key_lo - j * BN, c_hi = key_hi - j * BN;
 #pragma unroll
           for (int c = 0; c < BN; ++c) s[c] = (c >= c_lo && c <= c_hi) ? s[c] : -INFINITY;
         }
-        float mx = fmax3(s[0], s[1], s[2]);
+        // row maximum: four independent chains of three-input max
+        float mc[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-        for (int c = 3; c < BN - 1; c += 2) mx = fmax3(mx, s[c], s[c + 1]);
-        mx = fmaxf(mx, s[BN - 1]);
+        for (int c = 4; c < BN; c += 8)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) mc[q] = fmax3(mc[q], s[c + 2 * q], s[c + 2 * q + 1]);
+        const float mx = fmaxf(fmax3(mc[0], mc[1], mc[2]), mc[3]);
         const float m_tile = mx * p.scale_log2;
         float alpha = 1.f;
         if (m_tile > m_ref + kTau) {
           alpha = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - m_tile);
           l *= alpha;
           m_ref = m_tile;
+        }
+        if constexpr (C::SEP_P) {
+          // P_i(j-1) V must be complete before O_i is rescaled or P_i rewritten
+          if (j > my_lo) {
+            ok = mbar_wait(&o_done[i], pv & 1, abort_flag, p.err);
+            ++pv;
+            if (!__all_sync(0xffffffffu, ok)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
         }
         const bool rescale = (j > my_lo) && (alpha != 1.f);
         if (__any_sync(0xffffffffu, rescale)) {
@@ -407,34 +534,52 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float mb = (m_ref == -INFINITY) ? 0.f : m_ref;
         const uint64_t nm2 = f2_pack(-mb, -mb);
         uint32_t pk[BN / 2];
-        uint64_t sum2 = f2_pack(0.f, 0.f);
+        uint64_t sum2[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) sum2[q] = f2_pack(0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < BN; c += 2) {
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), c2, nm2), x0, x1);
-          const float p0 = ex2(x0), p1 = ex2(x1);
-          sum2 = f2_add(sum2, f2_pack(p0, p1));
+          const uint64_t x2 = f2_fma(f2_pack(s[c], s[c + 1]), c2, nm2);
+          float p0, p1;
+          if ((c / 2) % 16 < kEmuPer16) {
+            f2_unpack(exp2_fma2(x2), p0, p1);
+          } else {
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            p0 = ex2(x0);
+            p1 = ex2(x1);
+          }
+          sum2[(c / 2) % 4] = f2_add(sum2[(c / 2) % 4], f2_pack(p0, p1));
           pk[c / 2] = pack_bf16x2(p0, p1);
         }
-        float s0, s1;
-        f2_unpack(sum2, s0, s1);
-        l += s0 + s1;
+        float s0, s1, s2, s3;
+        f2_unpack(f2_add(sum2[0], sum2[1]), s0, s1);
+        f2_unpack(f2_add(sum2[2], sum2[3]), s2, s3);
+        l += (s0 + s1) + (s2 + s3);
 #pragma unroll
-        for (int c = 0; c < BN / 64; ++c) tmem_st32(s_tmem + 32 * c, pk + 32 * c);
+        for (int c = 0; c < BN / 64; ++c) tmem_st32(p_tmem + 32 * c, pk + 32 * c);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&p_ready[i]);
       }
       if (!ok) break;
       // ---- epilogue: O / l -> bf16 (tcgen05.ld is warp-collective: every lane loads)
-      ok = mbar_wait(&o_done[i], oc & 1, abort_flag, p.err);
-      ++oc;
+      if constexpr (C::SEP_P) {
+        ok = mbar_wait(&o_done[i], pv & 1, abort_flag, p.err);
+        ++pv;
+      } else {
+        ok = mbar_wait(&o_done[i], oc & 1, abort_flag, p.err);
+        ++oc;
+      }
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      // a row with no visible key is 0 (the FMA-pipe exp2 maps masked scores
+      // to about 2^-126 instead of exactly 0)
+      const bool has_keys = key_hi >= max(key_lo, 0);
+      const float inv = (has_keys && l > 0.f) ? 1.f / l : 0.f;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
