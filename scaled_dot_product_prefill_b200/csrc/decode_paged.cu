@@ -43,6 +43,17 @@ namespace {
 constexpr int kWarps = 4;       // warps per split CTA
 constexpr int kChunk = 16;      // tokens per chunk (one bulk copy per K and per V)
 constexpr float kTau = 8.0f;    // lazy-rescale threshold, log2 units
+// Ring depth per warp (16-token K+V chunks at D = 128; twice as many at D = 64)
+// and the CTAs per SM the register allocation aims for.
+#ifndef ATTN_DECODE_STAGES
+#define ATTN_DECODE_STAGES 2
+#endif
+#ifndef ATTN_DECODE_SPLIT
+#define ATTN_DECODE_SPLIT 512
+#endif
+#ifndef ATTN_DECODE_MINB
+#define ATTN_DECODE_MINB 3
+#endif
 
 struct DecodeParams {
   const __nv_bfloat16* q;
@@ -59,13 +70,11 @@ struct DecodeParams {
   float scale_log2;
 };
 
-__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
+// 8 bf16 (one 16-byte load) as 4 packed fp32 pairs (element 2i in the low half).
+__device__ __forceinline__ void bf16x8_to_f2(const uint4& u, uint64_t (&f)[4]) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
+  for (int i = 0; i < 4; ++i) f[i] = f2_pack(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
 }
 
 // Sum NV per-lane values over groups of R lanes (lane bits below R) and
@@ -102,7 +111,7 @@ struct Geo {
   static constexpr int TPL = 32 / R;              // tokens per warp-wide 16 B load
   static constexpr int NL = kChunk / TPL;         // loads per chunk per lane
   static constexpr int CHUNK_BYTES = kChunk * D * 2;
-  static constexpr int STAGES = (D == 128) ? 3 : 4;
+  static constexpr int STAGES = (D == 128) ? ATTN_DECODE_STAGES : 2 * ATTN_DECODE_STAGES;
 };
 
 template <int D, int G>
@@ -116,7 +125,7 @@ struct SplitSmem {
 };
 
 template <int D, int G>
-__global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kWarps * 32, ATTN_DECODE_MINB) decode_split_kernel(const DecodeParams p) {
   using Gm = Geo<D>;
   constexpr int R = Gm::R, TPL = Gm::TPL, NL = Gm::NL, STAGES = Gm::STAGES;
   constexpr int NV = NL * G;                       // partial dot products per lane per chunk
@@ -185,23 +194,26 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(const DecodeP
 
   // query of the G heads of this group, my 8 columns, pre-scaled to log2 units
   const int d0 = (lane % R) * 8;
-  float qf[G][8];
+  // (packed fp32 pairs: the dot products and the P.V accumulation run as f32x2 FMAs)
+  uint64_t q2[G][4];
+  const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
 #pragma unroll
   for (int hh = 0; hh < G; ++hh) {
     const uint4 u = *reinterpret_cast<const uint4*>(
         p.q + (static_cast<size_t>(b) * p.Hq + g * G + hh) * D + d0);
-    bf16x8_to_f32(u, qf[hh]);
+    bf16x8_to_f2(u, q2[hh]);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) qf[hh][e] *= p.scale_log2;
+    for (int e = 0; e < 4; ++e) q2[hh][e] = f2_mul(q2[hh][e], sc2);
   }
 
-  float m_ref[G], l_part[G], acc[G][8];
+  float m_ref[G], l_part[G];
+  uint64_t acc2[G][4];
 #pragma unroll
   for (int hh = 0; hh < G; ++hh) {
     m_ref[hh] = -INFINITY;
     l_part[hh] = 0.f;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[hh][e] = 0.f;
+    for (int e = 0; e < 4; ++e) acc2[hh][e] = f2_pack(0.f, 0.f);
   }
 
   bool ok_all = true;
@@ -224,14 +236,16 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(const DecodeP
     float part[NV];
 #pragma unroll
     for (int l = 0; l < NL; ++l) {
-      float kf[8];
-      bf16x8_to_f32(sk[l * 32 + lane], kf);
+      uint64_t k2[4];
+      bf16x8_to_f2(sk[l * 32 + lane], k2);
 #pragma unroll
       for (int hh = 0; hh < G; ++hh) {
-        float a = 0.f;
+        uint64_t a = f2_mul(q2[hh][0], k2[0]);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) a = fmaf(qf[hh][e], kf[e], a);
-        part[l * G + hh] = a;
+        for (int e = 1; e < 4; ++e) a = f2_fma(q2[hh][e], k2[e], a);
+        float x0, x1;
+        f2_unpack(a, x0, x1);
+        part[l * G + hh] = x0 + x1;
       }
     }
     int base;
@@ -266,8 +280,9 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(const DecodeP
         if (mx > m_ref[hh] + kTau) {
           const float alpha = (m_ref[hh] == -INFINITY) ? 0.f : ex2(m_ref[hh] - mx);
           l_part[hh] *= alpha;
+          const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) acc[hh][e] *= alpha;
+          for (int e = 0; e < 4; ++e) acc2[hh][e] = f2_mul(acc2[hh][e], a2);
           m_ref[hh] = mx;
         }
       }
@@ -298,15 +313,15 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(const DecodeP
         const int t = chunk_t0 + tok;
         if (!(stage_ok && t >= lo && t < L)) u = make_uint4(0u, 0u, 0u, 0u);  // poisoned slots stay out
       }
-      float vf[8];
-      bf16x8_to_f32(u, vf);
-      float pv[G];
+      uint64_t v2[4];
+      bf16x8_to_f2(u, v2);
 #pragma unroll
-      for (int hh = 0; hh < G; ++hh) pv[hh] = pb[tok * G + hh];
+      for (int hh = 0; hh < G; ++hh) {
+        const float pr = pb[tok * G + hh];
+        const uint64_t pp = f2_pack(pr, pr);
 #pragma unroll
-      for (int hh = 0; hh < G; ++hh)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[hh][e] = fmaf(pv[hh], vf[e], acc[hh][e]);
+        for (int e = 0; e < 4; ++e) acc2[hh][e] = f2_fma(pp, v2[e], acc2[hh][e]);
+      }
     }
     __syncwarp();
     fence_proxy_async_smem();
@@ -314,6 +329,11 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(const DecodeP
   }
 
   // ---- per-warp totals: accumulators over the TPL token groups, sums over all lanes
+  float acc[G][8];
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) f2_unpack(acc2[hh][e], acc[hh][2 * e], acc[hh][2 * e + 1]);
 #pragma unroll
   for (int hh = 0; hh < G; ++hh) {
 #pragma unroll
@@ -423,9 +443,10 @@ DecodeGeometry decode_geometry(int N, int Hq, int D, int max_seq_len, int page_s
   (void)D;
   (void)page_size;
   DecodeGeometry g{};
-  // 512 keys per split: 8 chunks per warp, enough to amortise the pipeline
-  // fill; shorter splits when the batch is too small to fill the GPU.
-  int split = 512;
+  // ATTN_DECODE_SPLIT keys per split (8 chunks per warp at 512), enough to
+  // amortise the pipeline fill; shorter splits when the batch is too small
+  // to fill the GPU.
+  int split = ATTN_DECODE_SPLIT;
   const long long units = static_cast<long long>(N);
   while (split > 64 && units * ((max_seq_len + split - 1) / split) < 1024) split /= 2;
   g.split_tokens = split;
