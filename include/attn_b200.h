@@ -111,6 +111,23 @@ attn_status_t attn_prefill(const void* q, const void* k, const void* v, void* ou
                            float scale, int causal, int window, attn_stream_t stream);
 
 /*
+ * attn_prefill_lse -- attn_prefill that also returns the log-sum-exp of every
+ * query row ("Attention From Scratch" README, section "Quick start": the
+ * Flash Attention module returns (output, lse)):
+ *
+ *     lse[b, h, i] = log( sum over visible j of exp(q_i . k_j * scale) )
+ *
+ * natural logarithm, fp32; -inf for a row with no visible key.  With it,
+ * attention over two disjoint key sets can be merged exactly:
+ * O = (e^lse1 O1 + e^lse2 O2) / (e^lse1 + e^lse2).
+ * lse : [B, Hq, Sq] float, 4-byte aligned, device; must not be null.
+ * Everything else as attn_prefill.
+ */
+attn_status_t attn_prefill_lse(const void* q, const void* k, const void* v, void* out, float* lse,
+                               int B, int Hq, int Hkv, int Sq, int Skv, int D,
+                               float scale, int causal, int window, attn_stream_t stream);
+
+/*
  * attn_prefill_f32 -- the same operation with fp32 inputs and output, fp32
  * arithmetic throughout (FFMA on the CUDA cores; no TF32), for results
  * that must agree with a float64 evaluation to about 1e-5.
@@ -121,6 +138,11 @@ attn_status_t attn_prefill(const void* q, const void* k, const void* v, void* ou
 attn_status_t attn_prefill_f32(const float* q, const float* k, const float* v, float* out,
                                int B, int Hq, int Hkv, int Sq, int Skv, int D,
                                float scale, int causal, int window, attn_stream_t stream);
+
+/* attn_prefill_f32 with the per-row log-sum-exp, as attn_prefill_lse. */
+attn_status_t attn_prefill_f32_lse(const float* q, const float* k, const float* v, float* out, float* lse,
+                                   int B, int Hq, int Hkv, int Sq, int Skv, int D,
+                                   float scale, int causal, int window, attn_stream_t stream);
 
 /*
  * attn_decode_paged -- one decode step for N sequences over a paged KV cache.

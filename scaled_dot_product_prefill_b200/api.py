@@ -13,7 +13,8 @@ import torch
 from . import _lib
 from ._lib import AttnError
 
-__all__ = ["attn_prefill", "attn_prefill_f32", "attn_decode_paged", "attn_decode_paged_noalloc",
+__all__ = ["attn_prefill", "attn_prefill_f32", "attn_prefill_lse", "attn_prefill_f32_lse",
+           "attn_decode_paged", "attn_decode_paged_noalloc",
            "attn_decode_paged_workspace_size",
            "attn_device_status", "attn_status_string", "attn_version", "AttnError"]
 
@@ -79,6 +80,34 @@ def attn_prefill(q, k, v, *, causal=False, window=0, scale=None, out=None, strea
 def attn_prefill_f32(q, k, v, *, causal=False, window=0, scale=None, out=None, stream=None):
     """fp32 prefill (CUDA-core kernel), same layouts as attn_prefill."""
     return _prefill("attn_prefill_f32", torch.float32, q, k, v, causal, window, scale, out, stream)
+
+
+def _prefill_lse(name, dtype, q, k, v, causal, window, scale, out, lse, stream):
+    if q.dtype != dtype or k.dtype != dtype or v.dtype != dtype:
+        raise ValueError(f"{name} expects {dtype} q, k, v")
+    B, Hq, Sq, D = q.shape
+    _, Hkv, Skv, _ = k.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    _need_cuda(q, k, v, out, lse)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    fn = getattr(_lib.load(), name)
+    _check(name, fn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Skv, D, float(scale),
+                    int(bool(causal)), int(window), _stream(stream)))
+    return out, lse
+
+
+def attn_prefill_lse(q, k, v, *, causal=False, window=0, scale=None, out=None, lse=None, stream=None):
+    """bf16 prefill returning (out, lse); lse [B,Hq,Sq] fp32 natural-log log-sum-exp per row."""
+    return _prefill_lse("attn_prefill_lse", torch.bfloat16, q, k, v, causal, window, scale, out, lse, stream)
+
+
+def attn_prefill_f32_lse(q, k, v, *, causal=False, window=0, scale=None, out=None, lse=None, stream=None):
+    """fp32 prefill returning (out, lse)."""
+    return _prefill_lse("attn_prefill_f32_lse", torch.float32, q, k, v, causal, window, scale, out, lse, stream)
 
 
 def attn_decode_paged_workspace_size(N, Hq, D, max_seq_len, page_size) -> int:

@@ -32,6 +32,24 @@ unsigned int* device_error_word() {
 
 }  // namespace attn
 
+namespace attn {
+namespace {
+__global__ void fill_neg_inf_kernel(float* p, size_t n) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    p[i] = -INFINITY;
+}
+}  // namespace
+
+cudaError_t fill_neg_inf(float* p, size_t n, cudaStream_t stream) {
+  if (n == 0) return cudaSuccess;
+  const size_t want = (n + 255) / 256;
+  const unsigned blocks = static_cast<unsigned>(want < 4096 ? want : 4096);
+  fill_neg_inf_kernel<<<blocks, 256, 0, stream>>>(p, n);
+  return cudaGetLastError();
+}
+}  // namespace attn
+
 namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -70,29 +88,69 @@ const char* attn_status_string(attn_status_t s) {
   return "ATTN_ERR_UNKNOWN";
 }
 
-int attn_version(void) { return 100; }
+int attn_version(void) { return 101; }
+
+}  // extern "C"
+
+namespace {
+
+attn_status_t prefill_bf16(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
+                           int Hkv, int Sq, int Skv, int D, float scale, int causal, int window,
+                           attn_stream_t stream) {
+  const attn_status_t st = check_prefill(q, k, v, out, B, Hq, Hkv, Sq, Skv, D, scale, causal, window);
+  if (st != ATTN_OK || B == 0 || Hq == 0 || Sq == 0) return st;
+  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (Skv == 0) {  // no key at all: every row is empty, its output 0 and its lse -inf
+    if (cudaMemsetAsync(out, 0, static_cast<size_t>(B) * Hq * Sq * D * 2, s) != cudaSuccess) return ATTN_ERR_CUDA;
+    return lse == nullptr ? ATTN_OK : from_cuda(attn::fill_neg_inf(lse, static_cast<size_t>(B) * Hq * Sq, s));
+  }
+  return from_cuda(attn::launch_prefill_tc(q, k, v, out, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal, window,
+                                           attn::device_error_word(), s));
+}
+
+attn_status_t prefill_f32(const float* q, const float* k, const float* v, float* out, float* lse, int B, int Hq,
+                          int Hkv, int Sq, int Skv, int D, float scale, int causal, int window,
+                          attn_stream_t stream) {
+  const attn_status_t st = check_prefill(q, k, v, out, B, Hq, Hkv, Sq, Skv, D, scale, causal, window);
+  if (st != ATTN_OK || B == 0 || Hq == 0 || Sq == 0) return st;
+  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * Hq > 65535) return ATTN_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (Skv == 0) {
+    if (cudaMemsetAsync(out, 0, static_cast<size_t>(B) * Hq * Sq * D * sizeof(float), s) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    return lse == nullptr ? ATTN_OK : from_cuda(attn::fill_neg_inf(lse, static_cast<size_t>(B) * Hq * Sq, s));
+  }
+  return from_cuda(attn::launch_prefill_f32(q, k, v, out, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal, window, s));
+}
+
+}  // namespace
+
+extern "C" {
 
 attn_status_t attn_prefill(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv, int Sq,
                            int Skv, int D, float scale, int causal, int window, attn_stream_t stream) {
-  const attn_status_t st = check_prefill(q, k, v, out, B, Hq, Hkv, Sq, Skv, D, scale, causal, window);
-  if (st != ATTN_OK || B == 0 || Hq == 0 || Sq == 0) return st;
-  if (Skv == 0)  // no key at all: every row is empty and its output is 0
-    return from_cuda(cudaMemsetAsync(out, 0, static_cast<size_t>(B) * Hq * Sq * D * 2,
-                                     reinterpret_cast<cudaStream_t>(stream)));
-  return from_cuda(attn::launch_prefill_tc(q, k, v, out, B, Hq, Hkv, Sq, Skv, D, scale, causal, window,
-                                           attn::device_error_word(), reinterpret_cast<cudaStream_t>(stream)));
+  return prefill_bf16(q, k, v, out, nullptr, B, Hq, Hkv, Sq, Skv, D, scale, causal, window, stream);
+}
+
+attn_status_t attn_prefill_lse(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
+                               int Hkv, int Sq, int Skv, int D, float scale, int causal, int window,
+                               attn_stream_t stream) {
+  if (lse == nullptr && B > 0 && Hq > 0 && Sq > 0) return ATTN_ERR_INVALID_ARG;
+  return prefill_bf16(q, k, v, out, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal, window, stream);
 }
 
 attn_status_t attn_prefill_f32(const float* q, const float* k, const float* v, float* out, int B, int Hq, int Hkv,
                                int Sq, int Skv, int D, float scale, int causal, int window, attn_stream_t stream) {
-  const attn_status_t st = check_prefill(q, k, v, out, B, Hq, Hkv, Sq, Skv, D, scale, causal, window);
-  if (st != ATTN_OK || B == 0 || Hq == 0 || Sq == 0) return st;
-  if (static_cast<long long>(B) * Hq > 65535) return ATTN_ERR_UNSUPPORTED;
-  if (Skv == 0)
-    return from_cuda(cudaMemsetAsync(out, 0, static_cast<size_t>(B) * Hq * Sq * D * sizeof(float),
-                                     reinterpret_cast<cudaStream_t>(stream)));
-  return from_cuda(attn::launch_prefill_f32(q, k, v, out, B, Hq, Hkv, Sq, Skv, D, scale, causal, window,
-                                            reinterpret_cast<cudaStream_t>(stream)));
+  return prefill_f32(q, k, v, out, nullptr, B, Hq, Hkv, Sq, Skv, D, scale, causal, window, stream);
+}
+
+attn_status_t attn_prefill_f32_lse(const float* q, const float* k, const float* v, float* out, float* lse, int B,
+                                   int Hq, int Hkv, int Sq, int Skv, int D, float scale, int causal, int window,
+                                   attn_stream_t stream) {
+  if (lse == nullptr && B > 0 && Hq > 0 && Sq > 0) return ATTN_ERR_INVALID_ARG;
+  return prefill_f32(q, k, v, out, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal, window, stream);
 }
 
 size_t attn_decode_paged_workspace_size(int N, int Hq, int D, int max_seq_len, int page_size) {

@@ -24,12 +24,16 @@ __device__ __forceinline__ void record_error(unsigned int* err, unsigned int bit
 // Device address of this device's error word (looked up once per device).
 unsigned int* device_error_word();
 
+// Write -inf to n floats (the log-sum-exp of rows with no visible key).
+cudaError_t fill_neg_inf(float* p, size_t n, cudaStream_t stream);
+
 // Host-side launchers (defined next to their kernels).
-cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv,
-                              int Sq, int Skv, int D, float scale, int causal, int window,
+// lse (optional, may be null): [B, Hq, Sq] float, natural-log log-sum-exp of each row's scaled scores.
+cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
+                              int Hkv, int Sq, int Skv, int D, float scale, int causal, int window,
                               unsigned int* err, cudaStream_t stream);
-cudaError_t launch_prefill_f32(const float* q, const float* k, const float* v, float* out, int B, int Hq,
-                               int Hkv, int Sq, int Skv, int D, float scale, int causal, int window,
+cudaError_t launch_prefill_f32(const float* q, const float* k, const float* v, float* out, float* lse, int B,
+                               int Hq, int Hkv, int Sq, int Skv, int D, float scale, int causal, int window,
                                cudaStream_t stream);
 
 struct DecodeGeometry {

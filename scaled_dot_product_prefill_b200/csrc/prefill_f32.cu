@@ -23,7 +23,8 @@ template <int D>
 __global__ void __launch_bounds__(kRows * 32) prefill_f32_kernel(const float* __restrict__ q,
                                                                   const float* __restrict__ k,
                                                                   const float* __restrict__ v,
-                                                                  float* __restrict__ out, int Hq, int Hkv,
+                                                                  float* __restrict__ out,
+                                                                  float* __restrict__ lse, int Hq, int Hkv,
                                                                   int Sq, int Skv, float scale_log2,
                                                                   int causal, int window) {
   constexpr int PER = D / 32;            // output columns per lane
@@ -108,6 +109,8 @@ __global__ void __launch_bounds__(kRows * 32) prefill_f32_kernel(const float* __
 
   if (row < Sq) {
     const float inv = (l > 0.f) ? 1.f / l : 0.f;
+    if (lse != nullptr && lane == 0)   // log(sum_j exp(s_ij * scale)) = (m + log2 l) * ln 2
+      lse[static_cast<size_t>(bh) * Sq + row] = (l > 0.f) ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
     float* op = out + (static_cast<size_t>(bh) * Sq + row) * D;
 #pragma unroll
     for (int t = 0; t < PER; ++t) op[lane + 32 * t] = acc[t] * inv;
@@ -116,16 +119,17 @@ __global__ void __launch_bounds__(kRows * 32) prefill_f32_kernel(const float* __
 
 }  // namespace
 
-cudaError_t launch_prefill_f32(const float* q, const float* k, const float* v, float* out, int B, int Hq,
-                               int Hkv, int Sq, int Skv, int D, float scale, int causal, int window,
+cudaError_t launch_prefill_f32(const float* q, const float* k, const float* v, float* out, float* lse, int B,
+                               int Hq, int Hkv, int Sq, int Skv, int D, float scale, int causal, int window,
                                cudaStream_t stream) {
   const float scale_log2 = scale * 1.4426950408889634f;  // log2(e)
   dim3 grid((Sq + kRows - 1) / kRows, B * Hq);
   dim3 block(kRows * 32);
   if (D == 64) {
-    prefill_f32_kernel<64><<<grid, block, 0, stream>>>(q, k, v, out, Hq, Hkv, Sq, Skv, scale_log2, causal, window);
+    prefill_f32_kernel<64><<<grid, block, 0, stream>>>(q, k, v, out, lse, Hq, Hkv, Sq, Skv, scale_log2, causal,
+                                                       window);
   } else {
-    prefill_f32_kernel<128><<<grid, block, 0, stream>>>(q, k, v, out, Hq, Hkv, Sq, Skv, scale_log2, causal,
+    prefill_f32_kernel<128><<<grid, block, 0, stream>>>(q, k, v, out, lse, Hq, Hkv, Sq, Skv, scale_log2, causal,
                                                         window);
   }
   return cudaGetLastError();

@@ -91,6 +91,7 @@ struct Params {
   int B, Hq, Hkv, Sq, Skv, causal, window, n_qblocks, n_items;
   float scale_log2;
   __nv_bfloat16* out;
+  float* lse;           // [B, Hq, Sq] natural-log log-sum-exp, or null
   unsigned int* err;
 };
 
@@ -459,6 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (store) {
           uint4* dst = reinterpret_cast<uint4*>(orow);
           for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
+          if (p.lse != nullptr) p.lse[static_cast<size_t>(it.bh) * p.Sq + r] = -INFINITY;
         }
         continue;
       }
@@ -580,6 +582,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // to about 2^-126 instead of exactly 0)
       const bool has_keys = key_hi >= max(key_lo, 0);
       const float inv = (has_keys && l > 0.f) ? 1.f / l : 0.f;
+      if (p.lse != nullptr && store)   // log(sum_j exp(s_ij * scale)) = (m + log2 l) * ln 2
+        p.lse[static_cast<size_t>(it.bh) * p.Sq + r] =
+            (has_keys && l > 0.f) ? (m_ref + log2f(l)) * 0.6931471805599453f : -INFINITY;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -675,8 +680,8 @@ cudaError_t launch_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
 
 }  // namespace
 
-cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv,
-                              int Sq, int Skv, int D, float scale, int causal, int window, unsigned int* err,
+cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
+                              int Hkv, int Sq, int Skv, int D, float scale, int causal, int window, unsigned int* err,
                               cudaStream_t stream) {
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, q, D, Sq, B * Hq) || !make_map(&mk, k, D, Skv, B * Hkv) || !make_map(&mv, v, D, Skv, B * Hkv))
@@ -695,6 +700,7 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, void*
   p.n_items = static_cast<int>(items);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
   p.err = err;
   return D == 64 ? launch_d<64>(mq, mk, mv, p, stream) : launch_d<128>(mq, mk, mv, p, stream);
 }

@@ -123,3 +123,14 @@ def test_oracle_is_not_imported_by_the_library():
         if src and src.endswith(".py"):
             text = open(src).read()
             assert "import oracle" not in text and "from oracle" not in text, src
+
+
+@pytest.mark.parametrize("fn", ["attn_prefill_lse", "attn_prefill_f32_lse"])
+def test_prefill_lse_argument_validation(fn):
+    lib = _lib()
+    call = lambda lse, **kw: getattr(lib, fn)(FAKE, FAKE, FAKE, FAKE, lse, kw.get("B", 1), 4, 2, 64, 64,
+                                              kw.get("D", 64), 0.125, 1, 0, None)
+    assert call(None) == 1                        # the lse output is required
+    assert call(ctypes.c_void_p(0x10002)) == 1    # misaligned lse
+    assert call(FAKE, D=96) == 2
+    assert call(None, B=0) == 0                   # empty problem

@@ -139,3 +139,51 @@ def test_repeated_calls_are_deterministic():
     a = run_prefill(inp, True, 0)
     b = run_prefill(inp, True, 0)
     assert torch.equal(a, b)
+
+
+LSE_CASES = [
+    (2, 4, 2, 300, 300, 128, True, 0),
+    (1, 2, 2, 700, 200, 64, True, 0),      # rows with no visible key: lse = -inf
+    (1, 2, 1, 520, 520, 64, True, 129),
+    (1, 4, 4, 256, 1000, 128, False, 0),
+]
+
+
+@pytest.mark.parametrize("shape", LSE_CASES, ids=[str(s) for s in LSE_CASES])
+def test_prefill_lse_matches_oracle(shape):
+    B, Hq, Hkv, Sq, Skv, D, causal, window = shape
+    inp = inputs.prefill_inputs(B, Hq, Hkv, Sq, Skv, D, seed=17)
+    out, lse = api.attn_prefill_lse(inp.q.cuda(), inp.k.cuda(), inp.v.cuda(), causal=causal, window=window)
+    torch.cuda.synchronize()
+    ref, ref_lse = sdpa.attention(inp.q, inp.k, inp.v, 1 / np.sqrt(D), causal, window, return_lse=True)
+    assert_parity(out, ref, "bf16", str(shape))
+    got = lse.cpu().double().numpy()
+    empty = np.isneginf(ref_lse)
+    assert np.array_equal(np.isneginf(got), empty)
+    # fp32 scores of exact bf16 products, ex2/log2 in fp32: 1e-3 absolute covers it with margin
+    assert np.abs(got[~empty] - ref_lse[~empty]).max() <= 1e-3
+    # the plain entry point writes the same output
+    plain = api.attn_prefill(inp.q.cuda(), inp.k.cuda(), inp.v.cuda(), causal=causal, window=window)
+    assert torch.equal(plain, out)
+
+
+def test_prefill_f32_lse_matches_oracle():
+    inp = inputs.prefill_inputs(1, 2, 2, 200, 333, 64, seed=8, dtype="f32")
+    out, lse = api.attn_prefill_f32_lse(inp.q.cuda(), inp.k.cuda(), inp.v.cuda(), causal=True, window=50)
+    torch.cuda.synchronize()
+    ref, ref_lse = sdpa.attention(inp.q, inp.k, inp.v, 0.125, True, 50, return_lse=True)
+    assert_parity(out, ref, "f32", "f32 lse case")
+    assert np.abs(lse.cpu().double().numpy() - ref_lse).max() <= 1e-4
+
+
+def test_lse_merges_two_key_halves_into_the_full_result():
+    """Attention over keys [0, n) equals the lse-weighted merge of [0, n/2) and [n/2, n) (non-causal)."""
+    inp = inputs.prefill_inputs(2, 4, 2, 384, 768, 128, seed=23)
+    q, k, v = inp.q.cuda(), inp.k.cuda(), inp.v.cuda()
+    full = api.attn_prefill(q, k, v)
+    o1, l1 = api.attn_prefill_lse(q, k[:, :, :384].contiguous(), v[:, :, :384].contiguous())
+    o2, l2 = api.attn_prefill_lse(q, k[:, :, 384:].contiguous(), v[:, :, 384:].contiguous())
+    m = torch.maximum(l1, l2)
+    w1, w2 = torch.exp(l1 - m)[..., None], torch.exp(l2 - m)[..., None]
+    merged = (w1 * o1.float() + w2 * o2.float()) / (w1 + w2)
+    assert (merged - full.float()).abs().max().item() <= 2e-2

@@ -310,3 +310,23 @@ def test_visible_pair_counts_match_the_oracle_predicate():
     # the sliding-window workload: min(i + 1, 4096) keys per query over 16384 queries
     assert workloads.visible_pairs(16384, 16384, True, 4096) == 58_722_304
     assert workloads.prefill_flops(workloads.WORKLOADS["gqa_swa_16k"]) == 4 * 128 * 32 * 58_722_304
+
+
+def test_lse_matches_python_log_sum_exp_and_merges_disjoint_key_sets():
+    """lse_i = log sum_j exp(s_ij) over visible keys (math.fsum in pure Python), -inf when none is visible;
+    merging two disjoint key sets by their lse reproduces attention over their union."""
+    q, k, v = rand(1, 2, 7, 4), rand(1, 2, 9, 4), rand(1, 2, 9, 4)
+    for causal, window in ((False, 0), (True, 0), (True, 3)):
+        _, lse = sdpa.attention(q, k, v, 0.6, causal, window, return_lse=True)
+        vis = sdpa.visible(7, 9, causal, window)
+        for h in range(2):
+            for i in range(7):
+                s = [0.6 * sum(q[0, h, i, d] * k[0, h, j, d] for d in range(4)) for j in range(9) if vis[i, j]]
+                want = math.log(math.fsum(math.exp(x) for x in s)) if s else -math.inf
+                assert lse[0, h, i] == pytest.approx(want, abs=1e-12)
+    o1, l1 = sdpa.attention(q, k[:, :, :4], v[:, :, :4], 0.6, False, return_lse=True)
+    o2, l2 = sdpa.attention(q, k[:, :, 4:], v[:, :, 4:], 0.6, False, return_lse=True)
+    full, lf = sdpa.attention(q, k, v, 0.6, False, return_lse=True)
+    w1, w2 = np.exp(l1 - lf)[..., None], np.exp(l2 - lf)[..., None]
+    np.testing.assert_allclose(w1 * o1 + w2 * o2, full, atol=1e-13)
+    np.testing.assert_allclose(np.logaddexp(l1, l2), lf, atol=1e-13)
