@@ -145,6 +145,42 @@ attn_status_t attn_prefill_f32_lse(const float* q, const float* k, const float* 
                                    float scale, int causal, int window, attn_stream_t stream);
 
 /*
+ * attn_prefill_paged -- bf16 prefill of a chunk of new tokens whose keys and
+ * values sit in a paged KV cache (chunked prefill: the cache pages of the
+ * "Attention From Scratch" README, section "Paged KV Cache", read by the
+ * tiled prefill of attn_prefill).
+ *
+ * q          : [B, Hq, Sq, D] bf16, the queries of the Sq newest tokens of
+ *              every sequence (the chunk being prefilled)
+ * k_pool     : [num_pages, Hkv, page_size, D] bf16; v_pool the same
+ * page_table : [B, max_pages] int32; entry p of row b holds tokens
+ *              [p*page_size, (p+1)*page_size) of sequence b
+ * seq_lens   : [B] int32 (device): tokens in each cache, the chunk's own
+ *              included (its K/V already appended); query i of sequence b
+ *              sits at position seq_lens[b] - Sq + i (bottom-right alignment)
+ * page_size  : 16, 32, 64, 128 or 256
+ * max_seq_len: host-side upper bound of seq_lens (longer sequences are
+ *              truncated and reported as ATTN_ERR_BAD_PAGE by attn_device_status)
+ * out        : [B, Hq, Sq, D] bf16;  lse: [B, Hq, Sq] float or NULL (as attn_prefill_lse)
+ * causal / window / scale / D: as attn_prefill (causal = 0 lets every query see
+ *              all seq_lens[b] keys).
+ * Whole pages are read: the slots of a sequence's last page past its final
+ * token must hold finite values (any finite content; it is masked out, but a
+ * NaN there would reach the output through 0 * NaN in P.V).  Pages that no
+ * sequence references are never read.  A page-table entry outside
+ * [0, num_pages) for a token that the sequence holds is never read: it is
+ * reported as ATTN_ERR_BAD_PAGE by attn_device_status and its keys
+ * contribute garbage instead.
+ * Errors: ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA.
+ */
+attn_status_t attn_prefill_paged(const void* q, const void* k_pool, const void* v_pool,
+                                 const int32_t* page_table, const int32_t* seq_lens,
+                                 int page_size, int B, int Hq, int Hkv, int Sq, int D,
+                                 int num_pages, int max_pages, int max_seq_len,
+                                 float scale, int causal, int window,
+                                 void* out, float* lse, attn_stream_t stream);
+
+/*
  * attn_decode_paged -- one decode step for N sequences over a paged KV cache.
  *
  * q          : [N, Hq, D] bf16, the new token's query of every sequence

@@ -8,4 +8,5 @@ library has not been built.
 from .api import (AttnError, attn_decode_paged, attn_decode_paged_noalloc,  # noqa: F401
                   attn_decode_paged_workspace_size,
                   attn_device_status, attn_prefill, attn_prefill_f32, attn_prefill_f32_lse, attn_prefill_lse,
+                  attn_prefill_paged,
                   attn_status_string, attn_version)

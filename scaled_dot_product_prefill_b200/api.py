@@ -14,7 +14,7 @@ from . import _lib
 from ._lib import AttnError
 
 __all__ = ["attn_prefill", "attn_prefill_f32", "attn_prefill_lse", "attn_prefill_f32_lse",
-           "attn_decode_paged", "attn_decode_paged_noalloc",
+           "attn_prefill_paged", "attn_decode_paged", "attn_decode_paged_noalloc",
            "attn_decode_paged_workspace_size",
            "attn_device_status", "attn_status_string", "attn_version", "AttnError"]
 
@@ -108,6 +108,31 @@ def attn_prefill_lse(q, k, v, *, causal=False, window=0, scale=None, out=None, l
 def attn_prefill_f32_lse(q, k, v, *, causal=False, window=0, scale=None, out=None, lse=None, stream=None):
     """fp32 prefill returning (out, lse)."""
     return _prefill_lse("attn_prefill_f32_lse", torch.float32, q, k, v, causal, window, scale, out, lse, stream)
+
+
+def attn_prefill_paged(q, k_pool, v_pool, page_table, seq_lens, *, max_seq_len, causal=True, window=0,
+                       scale=None, out=None, lse=None, want_lse=False, stream=None):
+    """Chunked prefill over a paged cache: q [B,Hq,Sq,D] are the last Sq tokens of each sequence.
+
+    Returns out, or (out, lse) with want_lse (or an lse tensor given).
+    """
+    B, Hq, Sq, D = q.shape
+    num_pages, Hkv, page_size, _ = k_pool.shape
+    max_pages = page_table.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    _need_cuda(q, k_pool, v_pool, page_table, seq_lens, out, lse)
+    if page_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise ValueError("page_table and seq_lens must be int32")
+    _check("attn_prefill_paged", _lib.load().attn_prefill_paged(
+        _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(page_table), _ptr(seq_lens), page_size, B, Hq, Hkv, Sq, D,
+        num_pages, max_pages, int(max_seq_len), float(scale), int(bool(causal)), int(window), _ptr(out), _ptr(lse),
+        _stream(stream)))
+    return (out, lse) if lse is not None else out
 
 
 def attn_decode_paged_workspace_size(N, Hq, D, max_seq_len, page_size) -> int:

@@ -141,6 +141,40 @@ attn_status_t attn_prefill_lse(const void* q, const void* k, const void* v, void
   return prefill_bf16(q, k, v, out, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal, window, stream);
 }
 
+attn_status_t attn_prefill_paged(const void* q, const void* k_pool, const void* v_pool, const int32_t* page_table,
+                                 const int32_t* seq_lens, int page_size, int B, int Hq, int Hkv, int Sq, int D,
+                                 int num_pages, int max_pages, int max_seq_len, float scale, int causal, int window,
+                                 void* out, float* lse, attn_stream_t stream) {
+  if (B < 0 || Hq < 0 || Hkv < 0 || Sq < 0 || D <= 0 || num_pages < 0 || max_pages < 0 || max_seq_len < 0 ||
+      window < 0 || page_size <= 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (B == 0 || Hq == 0 || Sq == 0) return ATTN_OK;
+  if (Hkv == 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (q == nullptr || out == nullptr || seq_lens == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (max_seq_len > 0 && (k_pool == nullptr || v_pool == nullptr || page_table == nullptr || max_pages == 0 ||
+                          num_pages == 0))
+    return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(page_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return ATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (window > 0 && !causal) return ATTN_ERR_UNSUPPORTED;
+  if (page_size != 16 && page_size != 32 && page_size != 64 && page_size != 128 && page_size != 256)
+    return ATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(num_pages) * Hkv > 0x7FFFFFFFLL) return ATTN_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (max_seq_len == 0) {  // every cache is empty: outputs 0, lse -inf
+    if (cudaMemsetAsync(out, 0, static_cast<size_t>(B) * Hq * Sq * D * 2, s) != cudaSuccess) return ATTN_ERR_CUDA;
+    return lse == nullptr ? ATTN_OK : from_cuda(attn::fill_neg_inf(lse, static_cast<size_t>(B) * Hq * Sq, s));
+  }
+  return from_cuda(attn::launch_prefill_tc_paged(q, k_pool, v_pool, page_table, seq_lens, page_size, B, Hq, Hkv, Sq,
+                                                 D, num_pages, max_pages, max_seq_len, scale, causal, window, out, lse,
+                                                 attn::device_error_word(), s));
+}
+
 attn_status_t attn_prefill_f32(const float* q, const float* k, const float* v, float* out, int B, int Hq, int Hkv,
                                int Sq, int Skv, int D, float scale, int causal, int window, attn_stream_t stream) {
   return prefill_f32(q, k, v, out, nullptr, B, Hq, Hkv, Sq, Skv, D, scale, causal, window, stream);

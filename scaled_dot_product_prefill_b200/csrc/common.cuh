@@ -32,6 +32,10 @@ cudaError_t fill_neg_inf(float* p, size_t n, cudaStream_t stream);
 cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
                               int Hkv, int Sq, int Skv, int D, float scale, int causal, int window,
                               unsigned int* err, cudaStream_t stream);
+cudaError_t launch_prefill_tc_paged(const void* q, const void* k_pool, const void* v_pool, const int32_t* page_table,
+                                    const int32_t* seq_lens, int page_size, int B, int Hq, int Hkv, int Sq, int D,
+                                    int num_pages, int max_pages, int max_seq_len, float scale, int causal,
+                                    int window, void* out, float* lse, unsigned int* err, cudaStream_t stream);
 cudaError_t launch_prefill_f32(const float* q, const float* k, const float* v, float* out, float* lse, int B,
                                int Hq, int Hkv, int Sq, int Skv, int D, float scale, int causal, int window,
                                cudaStream_t stream);

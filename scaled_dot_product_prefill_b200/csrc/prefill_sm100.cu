@@ -93,10 +93,16 @@ struct Params {
   __nv_bfloat16* out;
   float* lse;           // [B, Hq, Sq] natural-log log-sum-exp, or null
   unsigned int* err;
+  // paged K/V (paged != 0): K and V come from [num_pages, Hkv, page_size, D]
+  // pools through page_table [B, max_pages]; sequence b has seq_lens[b] keys
+  // (at most Skv, the caller's bound), and its Sq queries are the last Sq of them.
+  const int32_t* page_table;
+  const int32_t* seq_lens;
+  int paged, page_size, box_rows, max_pages, num_pages;
 };
 
 struct Item {
-  int bh, b, g, q_row0;
+  int bh, b, g, q_row0, skv;   // skv: keys of this item's sequence
   int lo[NQ], hi[NQ];   // key-tile range per query tile (empty if hi <= lo)
   int lo_all, hi_all;   // union; empty if hi_all <= lo_all
 };
@@ -116,8 +122,15 @@ __device__ __forceinline__ Item make_item(const Params& p, int k) {
   it.b = it.bh / p.Hq;
   it.g = (it.bh % p.Hq) / (p.Hq / p.Hkv);
   it.q_row0 = qb * (NQ * BM);
-  const int off = p.Skv - p.Sq;
-  const int n_kt = (p.Skv + BN - 1) / BN;
+  it.skv = p.Skv;
+  if (p.paged) {
+    const int L = p.seq_lens[it.b];
+    const int cap = min(p.Skv, p.max_pages * p.page_size);
+    if (L > cap) record_error(p.err, ATTN_ERRBIT_BADPAGE);
+    it.skv = max(0, min(L, cap));
+  }
+  const int off = it.skv - p.Sq;
+  const int n_kt = (it.skv + BN - 1) / BN;
   it.lo_all = 1 << 30;
   it.hi_all = 0;
 #pragma unroll
@@ -129,7 +142,7 @@ __device__ __forceinline__ Item make_item(const Params& p, int k) {
       if (!p.causal) {
         hi = n_kt;
       } else {
-        const int last_key = min(r1 - 1 + off, p.Skv - 1);
+        const int last_key = min(r1 - 1 + off, it.skv - 1);
         const int first_key = (p.window > 0) ? max(0, r0 + off - p.window + 1) : 0;
         if (last_key >= first_key && last_key >= 0) {
           lo = first_key / BN;
@@ -150,11 +163,12 @@ __device__ __forceinline__ Item make_item(const Params& p, int k) {
 
 __device__ __forceinline__ bool active(const Item& it, int i, int j) { return j >= it.lo[i] && j < it.hi[i]; }
 
-// True if every (row, key) pair of query rows [r0, r0+BM) x key tile j is visible.
-__device__ __forceinline__ bool tile_unmasked(const Params& p, int r0, int j) {
-  const int off = p.Skv - p.Sq;
+// True if every (row, key) pair of query rows [r0, r0+BM) x key tile j is visible
+// (skv keys in the sequence).
+__device__ __forceinline__ bool tile_unmasked(const Params& p, int skv, int r0, int j) {
+  const int off = skv - p.Sq;
   const int k0 = j * BN, k1 = j * BN + BN - 1;
-  if (k1 >= p.Skv) return false;
+  if (k1 >= skv) return false;
   if (!p.causal) return true;
   if (k1 > r0 + off) return false;
   if (p.window > 0 && k0 <= r0 + BM - 1 + off - p.window) return false;
@@ -246,8 +260,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(&empty[st], ((n / STAGES) & 1) ^ 1, abort_flag, p.err)) return false;
           mbar_arrive_expect_tx(&full[st], C::TILE_BYTES);
           const CUtensorMap* tm = is_v ? &tmap_v : &tmap_k;
-          for (int a = 0; a < C::KATOMS; ++a)
-            tma_load_3d(sRing + st * C::TILE_BYTES + a * BN * 128, tm, &full[st], a * 64, j * BN, kv_plane);
+          if (!p.paged) {
+            for (int a = 0; a < C::KATOMS; ++a)
+              tma_load_3d(sRing + st * C::TILE_BYTES + a * BN * 128, tm, &full[st], a * 64, j * BN, kv_plane);
+          } else {
+            // the key tile is assembled from page boxes of box_rows rows each; a
+            // box lands at its row offset inside the swizzled tile, so the MMA
+            // sees the same layout as a dense load
+            const int nb = BN / p.box_rows;
+            int phys[8];
+#pragma unroll
+            for (int rb = 0; rb < 8; ++rb) {
+              if (rb >= nb) break;
+              const int pg = (j * BN + rb * p.box_rows) / p.page_size;
+              phys[rb] = (pg < p.max_pages) ? p.page_table[static_cast<size_t>(it.b) * p.max_pages + pg] : -1;
+            }
+#pragma unroll
+            for (int rb = 0; rb < 8; ++rb) {
+              if (rb >= nb) break;
+              const int key0 = j * BN + rb * p.box_rows;
+              int ph = phys[rb];
+              if (ph < 0 || ph >= p.num_pages) {   // never read outside the pool
+                if (key0 < it.skv) record_error(p.err, ATTN_ERRBIT_BADPAGE);
+                ph = 0;                             // rows past the sequence end are masked
+              }
+              for (int a = 0; a < C::KATOMS; ++a)
+                tma_load_3d(sRing + st * C::TILE_BYTES + a * BN * 128 + rb * p.box_rows * 128, tm, &full[st],
+                            a * 64, key0 % p.page_size, ph * p.Hkv + it.g);
+            }
+          }
           ++n;
           return true;
         };
@@ -436,7 +477,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int i = warp >> 2;                 // query tile
     const int wq = warp & 3;                 // lane quarter of tensor memory
     const int rl = wq * 32 + lane;           // row within the tile
-    const int off = p.Skv - p.Sq;
     const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t s_tmem = tmem + lane_bits + C::S_COL + 128 * i;
     const uint32_t p_tmem = tmem + lane_bits + C::P_COL + C::P_STRIDE * i;
@@ -465,7 +505,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
       // visible keys of this row: [key_lo, key_hi]
-      const int key_hi = p.causal ? min(r + off, p.Skv - 1) : p.Skv - 1;
+      const int skv = it.skv;
+      const int off = skv - p.Sq;
+      const int key_hi = p.causal ? min(r + off, skv - 1) : skv - 1;
       const int key_lo = (p.causal && p.window > 0) ? r + off - p.window + 1 : 0;
       float m_ref = -INFINITY, l = 0.f;
 
@@ -484,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
           mbar_arrive(&s_free[i]);
         }
-        if (!tile_unmasked(p, r0, j)) {
+        if (!tile_unmasked(p, skv, r0, j)) {
           const int c_lo = key_lo - j * BN, c_hi = key_hi - j * BN;
 #pragma unroll
           for (int c = 0; c < BN; ++c) s[c] = (c >= c_lo && c <= c_hi) ? s[c] : -INFINITY;
@@ -631,14 +673,14 @@ EncodeTiledFn tensor_map_encoder() {
   return fn;
 }
 
-// [planes][rows][D] bf16 tensor, boxes of 64 columns x 128 rows, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, int D, int rows, int planes) {
+// [planes][rows][D] bf16 tensor, boxes of 64 columns x box_rows rows, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int D, int rows, int planes, int box_rows = 128) {
   EncodeTiledFn enc = tensor_map_encoder();
   if (enc == nullptr) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
                               static_cast<cuuint64_t>(planes)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(rows) * D * 2};
-  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -702,6 +744,41 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, void*
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
   p.err = err;
+  return D == 64 ? launch_d<64>(mq, mk, mv, p, stream) : launch_d<128>(mq, mk, mv, p, stream);
+}
+
+cudaError_t launch_prefill_tc_paged(const void* q, const void* k_pool, const void* v_pool, const int32_t* page_table,
+                                    const int32_t* seq_lens, int page_size, int B, int Hq, int Hkv, int Sq, int D,
+                                    int num_pages, int max_pages, int max_seq_len, float scale, int causal,
+                                    int window, void* out, float* lse, unsigned int* err, cudaStream_t stream) {
+  const int box_rows = page_size < BM ? page_size : BM;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, D, Sq, B * Hq) || !make_map(&mk, k_pool, D, page_size, num_pages * Hkv, box_rows) ||
+      !make_map(&mv, v_pool, D, page_size, num_pages * Hkv, box_rows))
+    return cudaErrorInvalidValue;
+  Params p{};
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Sq = Sq;
+  p.Skv = max_seq_len;
+  p.causal = causal;
+  p.window = window;
+  p.n_qblocks = (Sq + NQ * BM - 1) / (NQ * BM);
+  const long long items = static_cast<long long>(p.n_qblocks) * B * Hq;
+  if (items > (1LL << 30)) return cudaErrorInvalidValue;
+  p.n_items = static_cast<int>(items);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.err = err;
+  p.page_table = page_table;
+  p.seq_lens = seq_lens;
+  p.paged = 1;
+  p.page_size = page_size;
+  p.box_rows = box_rows;
+  p.max_pages = max_pages;
+  p.num_pages = num_pages;
   return D == 64 ? launch_d<64>(mq, mk, mv, p, stream) : launch_d<128>(mq, mk, mv, p, stream);
 }
 

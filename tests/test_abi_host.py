@@ -134,3 +134,18 @@ def test_prefill_lse_argument_validation(fn):
     assert call(ctypes.c_void_p(0x10002)) == 1    # misaligned lse
     assert call(FAKE, D=96) == 2
     assert call(None, B=0) == 0                   # empty problem
+
+
+def test_paged_prefill_argument_validation():
+    lib = _lib()
+
+    def call(page=16, D=128, lse=None, window=0, causal=1, Hq=8, Hkv=2, q=FAKE, msl=256):
+        return lib.attn_prefill_paged(q, FAKE, FAKE, FAKE, FAKE, page, 2, Hq, Hkv, 64, D, 64, 16, msl, 0.1, causal,
+                                      window, FAKE, lse, None)
+    assert call(q=None) == 1
+    assert call(Hq=8, Hkv=3) == 1
+    assert call(lse=ctypes.c_void_p(0x10002)) == 1
+    assert call(page=8) == 2
+    assert call(page=48) == 2
+    assert call(D=96) == 2
+    assert call(causal=0, window=16) == 2
