@@ -232,6 +232,8 @@ def run_ours(args, rank, world, local_rank):
     t_pre = [e[0].elapsed_time(e[1]) for e in evs]
     t_dec = [e[2].elapsed_time(e[3]) for e in evs]
     pre_ms, dec_ms = float(np.mean(t_pre)), float(np.mean(t_dec))
+    stats = {name: {"median": round(float(np.median(t)), 5), "mean": round(float(np.mean(t)), 5),
+                    "std": round(float(np.std(t)), 5)} for name, t in (("prefill_ms", t_pre), ("decode_ms", t_dec))}
     step_ms = pre_ms + dec_ms
     if dist is not None:
         tt = torch.tensor([pre_ms, dec_ms, step_ms], device=dev)
@@ -264,10 +266,17 @@ def run_ours(args, rank, world, local_rank):
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
     d2h = hout.numel() * hout.element_size()
 
+    # ---- the prefill replayed from a CUDA graph: the same kernel without the host launch path
+    graph_ms = None
+    if rank == 0 and not args.no_extra:
+        graph_ms = graph_prefill_ms(lambda: api.attn_prefill(q, k, v, causal=spec.causal, window=spec.window,
+                                                             scale=spec.scale, out=out), flush, args.steps)
+
     # ---- the other workloads, one line each (parity cases, reported for context)
     extra = {}
     if rank == 0 and not args.no_extra:
         extra = other_workloads(dev, peaks)
+        extra.update(append_workloads(dev, peaks))
 
     result = None
     if rank == 0:
@@ -303,7 +312,7 @@ def run_ours(args, rank, world, local_rank):
             },
             "roofline": {"bound": "tensor", "achieved": round(ach_t, 2), "peak": peak_t, "unit": "TFLOP/s",
                          "frac": round(ach_t / peak_t, 4), "traffic": traffic,
-                         "kernel": "prefill_tc_kernel<64>", "peak_kind": f"bf16 burst, {peak_kind}"},
+                         "kernel": "prefill_tc_kernel<64, false>", "peak_kind": f"bf16 burst, {peak_kind}"},
             "roofline_decode": {"bound": "hbm", "achieved": round(ach_d, 1), "peak": peak_h, "unit": "GB/s",
                                 "frac": round(ach_d / peak_h, 4), "traffic": traffic_d,
                                 "kernel": "decode_split_kernel<128,4> + decode_combine_kernel<128>",
@@ -311,6 +320,7 @@ def run_ours(args, rank, world, local_rank):
             "decode": {"value": round(world * d_bytes / (dec_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                        "ms": round(dec_ms, 5)},
             "prefill_ms": round(pre_ms, 5),
+            "timing": dict(stats, prefill_graph_ms=None if graph_ms is None else round(graph_ms, 5)),
             "e2e": {"value": round(world * p_flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms": round(e2e_ms, 5),
                     "path": "pinned host q/k/v -> device, attn_prefill, out -> pinned host"},
@@ -324,7 +334,7 @@ def run_ours(args, rank, world, local_rank):
     return result
 
 
-def time_call(fn, reps, flush=None):
+def time_call(fn, reps, flush=None, clean_flush=None):
     import torch
 
     for _ in range(3):
@@ -333,11 +343,77 @@ def time_call(fn, reps, flush=None):
     for e in ev:
         if flush is not None:
             flush.zero_()
+        if clean_flush is not None:
+            clean_flush.sum()
         e[0].record()
         fn()
         e[1].record()
     torch.cuda.synchronize()
     return float(np.median([a.elapsed_time(b) for a, b in ev]))
+
+
+def graph_prefill_ms(fn, flush, reps):
+    """Median time of fn replayed from a CUDA graph (captured once), with an L2 flush before each replay."""
+    import torch
+
+    reps = max(10, min(reps, 200))
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="relaxed"):
+        fn()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
+    for _ in range(3):
+        g.replay()
+    for e in ev:
+        flush.zero_()
+        e[0].record()
+        g.replay()
+        e[1].record()
+    torch.cuda.synchronize()
+    ms = float(np.median([a.elapsed_time(b) for a, b in ev]))
+    del g
+    return ms
+
+
+def append_workloads(dev, peaks):
+    """attn_kv_append on a decode step, a prefill chunk and a copy larger than L2.
+
+    HBM-bound copies: bytes = 2 (K, V) x 2 (read + write) x B x Hkv x S_new x D x 2 B.  The two serving
+    shapes run after a 256 MB read, which leaves L2 holding clean lines (a write flush would leave dirty
+    lines whose write-back lands inside the timed copy); the large one needs no flush.
+    """
+    import torch
+
+    from scaled_dot_product_prefill_b200 import api
+
+    clean = torch.ones(64 << 20, device=dev)
+    res = {}
+    shapes = {"kv_append_decode_step": (64, 8, 1, 128, 16, 4096, True),       # paged_decode_gqa's new tokens
+              "kv_append_prefill_chunk": (8, 12, 1024, 64, 16, 1024, True),   # mha_causal_gpt2s's K/V
+              "kv_append_large": (8, 8, 8192, 128, 16, 8192, False)}         # 537 MB moved, > L2
+    for name, (B, Hkv, S_new, D, page, L, flush) in shapes.items():
+        npg = -(-L // page)
+        perm = torch.randperm(B * npg, generator=torch.Generator().manual_seed(B)).to(torch.int32)
+        table = perm.reshape(B, npg).to(dev)
+        lens = torch.full((B,), L, dtype=torch.int32, device=dev)
+        kp = torch.zeros((B * npg, Hkv, page, D), dtype=torch.bfloat16, device=dev)
+        vp = torch.zeros_like(kp)
+        kn = torch.randn((B, Hkv, S_new, D), device=dev).to(torch.bfloat16)
+        vn = torch.randn_like(kn)
+        ms = time_call(lambda: api.attn_kv_append(kn, vn, kp, vp, table, lens), 50,
+                       clean_flush=clean if flush else None)
+        nbytes = 4 * B * Hkv * S_new * D * 2
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        res[name] = {"ms": round(ms, 5), "GB/s": round(gbs, 1), "bytes": nbytes,
+                     "frac_of_hbm": round(gbs / float(peaks["hbm_gbs"]), 4),
+                     "l2": "256 MB read before each call" if flush else "none (data > L2)"}
+        del kp, vp, kn, vn
+    torch.cuda.empty_cache()
+    return res
 
 
 def other_workloads(dev, peaks):

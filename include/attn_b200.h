@@ -79,7 +79,8 @@ typedef enum {
   ATTN_ERR_BAD_PAGE = 5,      /* a page-table entry was outside [0, num_pages), or a sequence was
                                  longer than max_pages * page_size or max_seq_len
                                  (reported by attn_device_status) */
-  ATTN_ERR_WORKSPACE = 6      /* workspace missing or smaller than attn_decode_paged_workspace_size */
+  ATTN_ERR_WORKSPACE = 6,     /* workspace missing or smaller than attn_decode_paged_workspace_size */
+  ATTN_ERR_OUT_OF_PAGES = 7   /* the page pool has too few free pages for a request (nothing changed) */
 } attn_status_t;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -164,10 +165,10 @@ attn_status_t attn_prefill_f32_lse(const float* q, const float* k, const float* 
  * out        : [B, Hq, Sq, D] bf16;  lse: [B, Hq, Sq] float or NULL (as attn_prefill_lse)
  * causal / window / scale / D: as attn_prefill (causal = 0 lets every query see
  *              all seq_lens[b] keys).
- * Whole pages are read: the slots of a sequence's last page past its final
- * token must hold finite values (any finite content; it is masked out, but a
- * NaN there would reach the output through 0 * NaN in P.V).  Pages that no
- * sequence references are never read.  A page-table entry outside
+ * Only the pages that hold a sequence's tokens are read; entries past its
+ * last page are never read.  The slots of the last page after the final
+ * token may hold anything, NaN included: they are masked, and their values
+ * are cleared before they reach the output.  A page-table entry outside
  * [0, num_pages) for a token that the sequence holds is never read: it is
  * reported as ATTN_ERR_BAD_PAGE by attn_device_status and its keys
  * contribute garbage instead.
@@ -261,6 +262,110 @@ size_t attn_decode_paged_workspace_size(int N, int Hq, int D, int max_seq_len, i
  * range, ATTN_ERR_CUDA if the read itself failed.  clear != 0 resets the word.
  */
 attn_status_t attn_device_status(int clear);
+
+/*
+ * ---------------------------------------------------------------------------
+ * Paged KV cache management: a host-side page pool and the append kernel.
+ *
+ * The "Attention From Scratch" README (section "Paged KV Cache") splits the
+ * cache into fixed-size pages held in one global pool, keeps a page table per
+ * sequence, and allocates and reclaims pages as sequences grow and finish;
+ * "LLM core technology" (section "PagedAttention") maps a sequence's logical
+ * blocks to non-contiguous physical blocks through that table.  Its "KV
+ * Cache" section, like the kv-cache walkthrough of "Taking LLMs apart (2)",
+ * appends the new token's k and v to the cache before the attention of that
+ * step.  The pool below manages the page ids and tables that attn_kv_append,
+ * attn_prefill_paged and attn_decode_paged consume; the K/V pools themselves
+ * are device memory the caller owns.
+ * ---------------------------------------------------------------------------
+ */
+
+/* Opaque host object.  It holds a free list of page ids 0..num_pages-1 and,
+ * for each sequence slot 0..max_seqs-1, its length in tokens and its page
+ * list (the row of the page table).  Not thread-safe: callers serialise. */
+typedef struct attn_page_pool attn_page_pool_t;
+
+/*
+ * attn_page_pool_create -- make a pool of num_pages pages of page_size tokens
+ * for up to max_seqs sequences of at most max_pages_per_seq pages each.  All
+ * pages start free and every sequence empty.  *pool receives the handle (host
+ * memory allocated by the library, released by attn_page_pool_destroy).
+ * Errors: ATTN_ERR_INVALID_ARG for a null handle pointer or a size <= 0.
+ */
+attn_status_t attn_page_pool_create(int num_pages, int page_size, int max_seqs, int max_pages_per_seq,
+                                    attn_page_pool_t** pool);
+
+/* Free the pool's host memory (NULL is a no-op).  Device copies made by
+ * attn_page_pool_upload are the caller's and stay valid. */
+void attn_page_pool_destroy(attn_page_pool_t* pool);
+
+/*
+ * attn_page_pool_resize -- set sequence `seq` to `len` tokens.  Growing takes
+ * ceil(len / page_size) - (pages held) pages from the free list and appends
+ * them to the sequence's page list; shrinking returns the pages past
+ * ceil(len / page_size) to the free list (the most recently freed page is
+ * the next one handed out).  Tokens already in the kept pages do not move.
+ * All or nothing: with too few free pages the call returns
+ * ATTN_ERR_OUT_OF_PAGES and changes nothing.
+ * Errors: ATTN_ERR_INVALID_ARG (null pool, seq out of range, len < 0 or
+ * more than max_pages_per_seq * page_size), ATTN_ERR_OUT_OF_PAGES.
+ */
+attn_status_t attn_page_pool_resize(attn_page_pool_t* pool, int seq, int len);
+
+/* attn_page_pool_release -- end sequence `seq`: all its pages go back to the
+ * free list and its length becomes 0 (resize to 0). */
+attn_status_t attn_page_pool_release(attn_page_pool_t* pool, int seq);
+
+/* Free pages left in the pool (-1 for a null pool). */
+int attn_page_pool_free_pages(const attn_page_pool_t* pool);
+
+/* Length in tokens of sequence `seq` (-1 for a null pool or seq out of range). */
+int attn_page_pool_seq_len(const attn_page_pool_t* pool, int seq);
+
+/*
+ * attn_page_pool_export -- copy the pool's state to HOST arrays:
+ * page_table [max_seqs, max_pages_per_seq] int32 (row s = the page ids of
+ * sequence s in token order, -1 after its last page) and seq_lens [max_seqs]
+ * int32.  Either pointer may be NULL to skip it.
+ */
+attn_status_t attn_page_pool_export(const attn_page_pool_t* pool, int32_t* page_table, int32_t* seq_lens);
+
+/*
+ * attn_page_pool_upload -- copy the rows changed since the last upload to the
+ * DEVICE arrays page_table [max_seqs, max_pages_per_seq] and seq_lens
+ * [max_seqs] (int32, laid out as attn_page_pool_export), with
+ * cudaMemcpyAsync on `stream`.  The first upload copies everything.  The
+ * copies read the pool's own pageable host memory, which the CUDA runtime
+ * stages before the call returns, so the pool may be changed right after.
+ * Kernels later on `stream` see the new tables.
+ * Errors: ATTN_ERR_INVALID_ARG (null pointer), ATTN_ERR_CUDA.
+ */
+attn_status_t attn_page_pool_upload(attn_page_pool_t* pool, int32_t* page_table, int32_t* seq_lens,
+                                    attn_stream_t stream);
+
+/*
+ * attn_kv_append -- write the keys and values of S_new new tokens of each of
+ * B sequences into the paged cache.
+ *
+ * k_new, v_new : [B, Hkv, S_new, D] bf16 (the k/v layout of attn_prefill;
+ *                one decode step is S_new = 1)
+ * k_pool, v_pool: [num_pages, Hkv, page_size, D] bf16, written in place
+ * page_table   : [B, max_pages] int32 (device)
+ * seq_lens     : [B] int32 (device), the cache lengths AFTER the append (the
+ *                array that attn_prefill_paged / attn_decode_paged then take):
+ *                token i of sequence b goes to position seq_lens[b] - S_new + i,
+ *                i.e. page page_table[b][pos / page_size], slot pos % page_size.
+ *                Positions below 0 (a cache shorter than the chunk) are skipped.
+ * page_size    : a multiple of 8 tokens; D a multiple of 8, at most 512.
+ * A position past max_pages * page_size, or a page-table entry outside
+ * [0, num_pages), writes nothing and is reported as ATTN_ERR_BAD_PAGE by
+ * attn_device_status.  The values are copied bit for bit.
+ * Errors: ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA.
+ */
+attn_status_t attn_kv_append(const void* k_new, const void* v_new, void* k_pool, void* v_pool,
+                             const int32_t* page_table, const int32_t* seq_lens,
+                             int page_size, int B, int Hkv, int S_new, int D,
+                             int num_pages, int max_pages, attn_stream_t stream);
 
 #ifdef __cplusplus
 }

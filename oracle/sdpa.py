@@ -163,6 +163,36 @@ def gather_pages(pool, page_table_row, seq_len: int, page_size: int) -> np.ndarr
     return out
 
 
+def append_pages(pool, page_table, seq_lens, new, page_size: int) -> np.ndarray:
+    """The paged cache after writing S_new new tokens of every sequence into it.
+
+    pool: [num_pages, Hkv, page_size, D]; new: [B, Hkv, S_new, D];
+    page_table [B, max_pages]; seq_lens [B] are the lengths AFTER the append.
+    Token i of sequence b is the cache's position p = seq_lens[b] - S_new + i
+    and goes to slot p % page_size of page page_table[b][p // page_size]
+    ([ANAT] "KV cache": the new token's k and v are stored before the step's
+    attention; [AFS] "Paged KV Cache": that store goes through the page table
+    into the shared pool).  Positions below 0 (a cache shorter than the chunk)
+    have no slot and are skipped.  Returns a new array in the pool's dtype;
+    every other slot keeps its value.
+    """
+    out = np.array(pool, copy=True)
+    new = np.asarray(new)
+    pt = np.asarray(page_table, dtype=np.int64)
+    B, Hkv, S_new, D = new.shape
+    for b in range(B):
+        L = int(seq_lens[b])
+        for i in range(S_new):
+            p = L - S_new + i
+            if p < 0:
+                continue
+            phys = pt[b, p // page_size]
+            if phys < 0 or phys >= out.shape[0]:
+                raise IndexError(f"page table entry {phys} for position {p} is outside the pool")
+            out[phys, :, p % page_size, :] = new[b, :, i, :]
+    return out
+
+
 def decode_paged(q, k_pool, v_pool, page_table, seq_lens, page_size: int, scale=None, window: int = 0):
     """One decode step per sequence over a paged KV cache.
 

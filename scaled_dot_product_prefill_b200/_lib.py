@@ -9,7 +9,7 @@ _lib = None
 
 ATTN_STATUS = {
     0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED", 3: "ATTN_ERR_CUDA",
-    4: "ATTN_ERR_TIMEOUT", 5: "ATTN_ERR_BAD_PAGE", 6: "ATTN_ERR_WORKSPACE",
+    4: "ATTN_ERR_TIMEOUT", 5: "ATTN_ERR_BAD_PAGE", 6: "ATTN_ERR_WORKSPACE", 7: "ATTN_ERR_OUT_OF_PAGES",
 }
 
 # name -> (restype, argtypes); mirrors include/attn_b200.h
@@ -27,6 +27,15 @@ PROTOTYPES = {
     "attn_decode_paged_noalloc": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 8 + [_c_float, _c_int, _vp, _vp]),
     "attn_decode_paged_workspace_size": (_c_size, [_c_int] * 5),
     "attn_device_status": (_c_int, [_c_int]),
+    "attn_kv_append": (_c_int, [_vp] * 6 + [_c_int] * 7 + [_vp]),
+    "attn_page_pool_create": (_c_int, [_c_int] * 4 + [ctypes.POINTER(_vp)]),
+    "attn_page_pool_destroy": (None, [_vp]),
+    "attn_page_pool_resize": (_c_int, [_vp, _c_int, _c_int]),
+    "attn_page_pool_release": (_c_int, [_vp, _c_int]),
+    "attn_page_pool_free_pages": (_c_int, [_vp]),
+    "attn_page_pool_seq_len": (_c_int, [_vp, _c_int]),
+    "attn_page_pool_export": (_c_int, [_vp, _vp, _vp]),
+    "attn_page_pool_upload": (_c_int, [_vp, _vp, _vp, _vp]),
 }
 
 

@@ -15,7 +15,7 @@ from ._lib import AttnError
 
 __all__ = ["attn_prefill", "attn_prefill_f32", "attn_prefill_lse", "attn_prefill_f32_lse",
            "attn_prefill_paged", "attn_decode_paged", "attn_decode_paged_noalloc",
-           "attn_decode_paged_workspace_size",
+           "attn_decode_paged_workspace_size", "attn_kv_append", "PagePool",
            "attn_device_status", "attn_status_string", "attn_version", "AttnError"]
 
 
@@ -190,3 +190,81 @@ def attn_decode_paged_noalloc(q, k_pool, v_pool, page_table, seq_lens, *, max_se
 def attn_device_status(clear: bool = True) -> int:
     """Status recorded by the kernels since the last clear (synchronises the device)."""
     return int(_lib.load().attn_device_status(int(bool(clear))))
+
+
+def attn_kv_append(k_new, v_new, k_pool, v_pool, page_table, seq_lens, *, stream=None):
+    """Write k_new/v_new [B,Hkv,S_new,D] into the pools at positions seq_lens[b] - S_new + i (seq_lens: after)."""
+    B, Hkv, S_new, D = k_new.shape
+    num_pages, Hkv_p, page_size, D_p = k_pool.shape
+    if tuple(v_new.shape) != tuple(k_new.shape) or tuple(v_pool.shape) != tuple(k_pool.shape):
+        raise ValueError("k_new/v_new and k_pool/v_pool must have matching shapes")
+    if Hkv_p != Hkv or D_p != D:
+        raise ValueError("the pools' head count and head dim must match k_new")
+    if k_new.dtype != torch.bfloat16 or v_new.dtype != torch.bfloat16 or k_pool.dtype != torch.bfloat16 \
+            or v_pool.dtype != torch.bfloat16:
+        raise ValueError("k_new, v_new and the pools must be bfloat16")
+    _need_cuda(k_new, v_new, k_pool, v_pool, page_table, seq_lens)
+    if page_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise ValueError("page_table and seq_lens must be int32")
+    _check("attn_kv_append", _lib.load().attn_kv_append(
+        _ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool), _ptr(page_table), _ptr(seq_lens), page_size, B, Hkv,
+        S_new, D, num_pages, page_table.shape[1], _stream(stream)))
+
+
+class PagePool:
+    """Host-side page allocator of the C ABI (attn_page_pool_*): page ids and per-sequence page tables.
+
+    ``resize(seq, len)`` grows or shrinks a sequence (all or nothing),
+    ``release(seq)`` returns its pages, ``export()`` gives host copies of the
+    table [max_seqs, max_pages_per_seq] and lengths [max_seqs], and
+    ``upload(page_table, seq_lens)`` copies the changed rows into device int32
+    tensors of those shapes on the current stream.
+    """
+
+    def __init__(self, num_pages, page_size, max_seqs, max_pages_per_seq):
+        import ctypes
+
+        self._lib = _lib.load()
+        handle = ctypes.c_void_p()
+        _check("attn_page_pool_create", self._lib.attn_page_pool_create(
+            int(num_pages), int(page_size), int(max_seqs), int(max_pages_per_seq), ctypes.byref(handle)))
+        self._h = handle
+        self.num_pages, self.page_size = int(num_pages), int(page_size)
+        self.max_seqs, self.max_pages_per_seq = int(max_seqs), int(max_pages_per_seq)
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            self._lib.attn_page_pool_destroy(self._h)
+        self._h = None
+
+    def __del__(self):
+        self.close()
+
+    def resize(self, seq, length):
+        _check("attn_page_pool_resize", self._lib.attn_page_pool_resize(self._h, int(seq), int(length)))
+
+    def release(self, seq):
+        _check("attn_page_pool_release", self._lib.attn_page_pool_release(self._h, int(seq)))
+
+    @property
+    def free_pages(self) -> int:
+        return int(self._lib.attn_page_pool_free_pages(self._h))
+
+    def seq_len(self, seq) -> int:
+        return int(self._lib.attn_page_pool_seq_len(self._h, int(seq)))
+
+    def export(self):
+        table = torch.empty((self.max_seqs, self.max_pages_per_seq), dtype=torch.int32)
+        lens = torch.empty((self.max_seqs,), dtype=torch.int32)
+        _check("attn_page_pool_export", self._lib.attn_page_pool_export(self._h, _ptr(table), _ptr(lens)))
+        return table, lens
+
+    def upload(self, page_table, seq_lens, stream=None):
+        if tuple(page_table.shape) != (self.max_seqs, self.max_pages_per_seq) or \
+                tuple(seq_lens.shape) != (self.max_seqs,):
+            raise ValueError("page_table must be [max_seqs, max_pages_per_seq] and seq_lens [max_seqs]")
+        if page_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+            raise ValueError("page_table and seq_lens must be int32")
+        _need_cuda(page_table, seq_lens)
+        _check("attn_page_pool_upload", self._lib.attn_page_pool_upload(
+            self._h, _ptr(page_table), _ptr(seq_lens), _stream(stream)))

@@ -1,4 +1,4 @@
-"""Build libattn_b200.so (all CUDA sources under csrc/) for sm_100a with nvcc.
+"""Build libattn_b200.so (the CUDA and C++ sources under csrc/) for sm_100a with nvcc.
 
 Each translation unit is compiled to an object under ``_build/`` (in
 parallel, skipped when up to date) and linked into
@@ -22,7 +22,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libattn_b200.so")
 
-SOURCES = ["attn_api.cu", "prefill_sm100.cu", "prefill_f32.cu", "decode_paged.cu"]
+SOURCES = ["attn_api.cu", "prefill_sm100.cu", "prefill_f32.cu", "decode_paged.cu", "kv_append.cu", "page_pool.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-I", INCLUDE, "-I", CSRC]

@@ -84,11 +84,12 @@ const char* attn_status_string(attn_status_t s) {
     case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT";
     case ATTN_ERR_BAD_PAGE: return "ATTN_ERR_BAD_PAGE";
     case ATTN_ERR_WORKSPACE: return "ATTN_ERR_WORKSPACE";
+    case ATTN_ERR_OUT_OF_PAGES: return "ATTN_ERR_OUT_OF_PAGES";
   }
   return "ATTN_ERR_UNKNOWN";
 }
 
-int attn_version(void) { return 101; }
+int attn_version(void) { return 102; }
 
 }  // extern "C"
 
@@ -164,7 +165,8 @@ attn_status_t attn_prefill_paged(const void* q, const void* k_pool, const void* 
   if (window > 0 && !causal) return ATTN_ERR_UNSUPPORTED;
   if (page_size != 16 && page_size != 32 && page_size != 64 && page_size != 128 && page_size != 256)
     return ATTN_ERR_UNSUPPORTED;
-  if (static_cast<long long>(num_pages) * Hkv > 0x7FFFFFFFLL) return ATTN_ERR_UNSUPPORTED;
+  // TMA plane coordinates (page * Hkv + g, one page past the pool for boxes past a sequence end) are int32
+  if ((static_cast<long long>(num_pages) + 1) * Hkv > 0x7FFFFFFFLL) return ATTN_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (max_seq_len == 0) {  // every cache is empty: outputs 0, lse -inf
     if (cudaMemsetAsync(out, 0, static_cast<size_t>(B) * Hq * Sq * D * 2, s) != cudaSuccess) return ATTN_ERR_CUDA;
@@ -235,6 +237,25 @@ attn_status_t attn_decode_paged_noalloc(const void* q, const void* k_pool, const
   }
   return attn_decode_paged(q, k_pool, v_pool, page_table, seq_lens, page_size, N, Hq, Hkv, D, num_pages, max_pages,
                            max_seq_len, scale, window, scratch, attn::decode_scratch_capacity(), out, stream);
+}
+
+attn_status_t attn_kv_append(const void* k_new, const void* v_new, void* k_pool, void* v_pool,
+                             const int32_t* page_table, const int32_t* seq_lens, int page_size, int B, int Hkv,
+                             int S_new, int D, int num_pages, int max_pages, attn_stream_t stream) {
+  if (B < 0 || Hkv < 0 || S_new < 0 || D <= 0 || page_size <= 0 || num_pages < 0 || max_pages < 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (B == 0 || Hkv == 0 || S_new == 0) return ATTN_OK;
+  if (k_new == nullptr || v_new == nullptr || k_pool == nullptr || v_pool == nullptr || page_table == nullptr ||
+      seq_lens == nullptr || num_pages == 0 || max_pages == 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_pool) || !aligned16(v_pool) ||
+      (reinterpret_cast<uintptr_t>(page_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+    return ATTN_ERR_INVALID_ARG;
+  if (D % 8 != 0 || D > 512 || page_size % 8 != 0) return ATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * Hkv * S_new * (D / 8) > 0x7FFFFFFFLL) return ATTN_ERR_UNSUPPORTED;
+  return from_cuda(attn::launch_kv_append(k_new, v_new, k_pool, v_pool, page_table, seq_lens, page_size, B, Hkv,
+                                          S_new, D, num_pages, max_pages, attn::device_error_word(),
+                                          reinterpret_cast<cudaStream_t>(stream)));
 }
 
 attn_status_t attn_device_status(int clear) {

@@ -93,12 +93,12 @@ struct Params {
   __nv_bfloat16* out;
   float* lse;           // [B, Hq, Sq] natural-log log-sum-exp, or null
   unsigned int* err;
-  // paged K/V (paged != 0): K and V come from [num_pages, Hkv, page_size, D]
+  // paged K/V (the PAGED kernels): K and V come from [num_pages, Hkv, page_size, D]
   // pools through page_table [B, max_pages]; sequence b has seq_lens[b] keys
   // (at most Skv, the caller's bound), and its Sq queries are the last Sq of them.
   const int32_t* page_table;
   const int32_t* seq_lens;
-  int paged, page_size, box_rows, max_pages, num_pages;
+  int page_size, box_rows, max_pages, num_pages;
 };
 
 struct Item {
@@ -114,6 +114,7 @@ __device__ __forceinline__ int item_index(const Params& p, int r) {
   return k < p.n_items ? k : -1;
 }
 
+template <bool PAGED>
 __device__ __forceinline__ Item make_item(const Params& p, int k) {
   Item it;
   const int BH = p.B * p.Hq;
@@ -123,7 +124,7 @@ __device__ __forceinline__ Item make_item(const Params& p, int k) {
   it.g = (it.bh % p.Hq) / (p.Hq / p.Hkv);
   it.q_row0 = qb * (NQ * BM);
   it.skv = p.Skv;
-  if (p.paged) {
+  if constexpr (PAGED) {
     const int L = p.seq_lens[it.b];
     const int cap = min(p.Skv, p.max_pages * p.page_size);
     if (L > cap) record_error(p.err, ATTN_ERRBIT_BADPAGE);
@@ -175,7 +176,10 @@ __device__ __forceinline__ bool tile_unmasked(const Params& p, int skv, int r0, 
   return true;
 }
 
-template <int D>
+// PAGED selects K/V through a page table (chunked prefill over a paged cache)
+// instead of dense [B, Hkv, Skv, D] tensors; the dense kernel carries none of
+// the paged code.
+template <int D, bool PAGED>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_v, const Params p) {
@@ -244,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int r = 0; r < n_rounds && ok; ++r) {
         const int k = item_index(p, r);
         if (k < 0) continue;
-        const Item it = make_item(p, k);
+        const Item it = make_item<PAGED>(p, k);
         if (it.hi_all <= it.lo_all) continue;
         const int qb = qn % QBUF;
         if (qn >= QBUF && !(ok = mbar_wait(&q_empty[qb], ((qn / QBUF) - 1) & 1, abort_flag, p.err))) break;
@@ -260,29 +264,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(&empty[st], ((n / STAGES) & 1) ^ 1, abort_flag, p.err)) return false;
           mbar_arrive_expect_tx(&full[st], C::TILE_BYTES);
           const CUtensorMap* tm = is_v ? &tmap_v : &tmap_k;
-          if (!p.paged) {
+          if constexpr (!PAGED) {
             for (int a = 0; a < C::KATOMS; ++a)
               tma_load_3d(sRing + st * C::TILE_BYTES + a * BN * 128, tm, &full[st], a * 64, j * BN, kv_plane);
           } else {
             // the key tile is assembled from page boxes of box_rows rows each; a
             // box lands at its row offset inside the swizzled tile, so the MMA
             // sees the same layout as a dense load
+            // boxes that start past the sequence end read no page: their plane
+            // coordinate is past the pool, so the copy fills them with zeros
             const int nb = BN / p.box_rows;
             int phys[8];
 #pragma unroll
             for (int rb = 0; rb < 8; ++rb) {
               if (rb >= nb) break;
-              const int pg = (j * BN + rb * p.box_rows) / p.page_size;
-              phys[rb] = (pg < p.max_pages) ? p.page_table[static_cast<size_t>(it.b) * p.max_pages + pg] : -1;
+              const int key0 = j * BN + rb * p.box_rows;
+              const int pg = key0 / p.page_size;
+              phys[rb] = (key0 < it.skv) ? p.page_table[static_cast<size_t>(it.b) * p.max_pages + pg] : 0;
             }
 #pragma unroll
             for (int rb = 0; rb < 8; ++rb) {
               if (rb >= nb) break;
               const int key0 = j * BN + rb * p.box_rows;
               int ph = phys[rb];
-              if (ph < 0 || ph >= p.num_pages) {   // never read outside the pool
-                if (key0 < it.skv) record_error(p.err, ATTN_ERRBIT_BADPAGE);
-                ph = 0;                             // rows past the sequence end are masked
+              if (key0 >= it.skv) {
+                ph = p.num_pages;                   // plane ph * Hkv + g is past the pool's planes
+              } else if (ph < 0 || ph >= p.num_pages) {   // never read outside the pool
+                record_error(p.err, ATTN_ERRBIT_BADPAGE);
+                ph = 0;
               }
               for (int a = 0; a < C::KATOMS; ++a)
                 tma_load_3d(sRing + st * C::TILE_BYTES + a * BN * 128 + rb * p.box_rows * 128, tm, &full[st],
@@ -336,6 +345,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(&s_ready[i]);
       };
+      // Paged K/V: the page box that holds a sequence's last key also brings the
+      // slots after it, whose contents are arbitrary.  Their scores are masked
+      // and P is 0 there, but 0 * NaN is NaN, so the V rows past the end are
+      // zeroed in shared memory before P.V reads them.  Boxes wholly past the
+      // end arrive as zeros already.
+      auto clear_v_tail = [&](int st, int j, int skv) {
+        if constexpr (!PAGED) return;
+        const int from = skv - j * BN;
+        if (from <= 0 || from >= BN) return;
+        const int to = min(BN, (from + p.box_rows - 1) / p.box_rows * p.box_rows);
+        if (to <= from) return;
+        for (int a = 0; a < C::KATOMS; ++a) {
+          const uint32_t base = smem_u32(sRing + st * C::TILE_BYTES + a * BN * 128);
+          for (int r = from; r < to; ++r)   // a 128-byte row holds the same key under the swizzle
+            for (int c = 0; c < 128; c += 16)
+              asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(base + r * 128 + c), "r"(0u)
+                           : "memory");
+        }
+        fence_proxy_async_smem();
+      };
       auto wait_slot = [&](int& st) -> bool {   // next ring slot, in load order
         st = n % STAGES;
         const bool r = mbar_wait(&full[st], (n / STAGES) & 1, abort_flag, p.err);
@@ -351,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int r = 0; r < n_rounds && ok; ++r) {
           const int k = item_index(p, r);
           if (k < 0) continue;
-          const Item it = make_item(p, k);
+          const Item it = make_item<PAGED>(p, k);
           if (it.hi_all <= it.lo_all) continue;
           const int qb = qn % QBUF;
           if (!(ok = mbar_wait(&q_full[qb], (qn / QBUF) & 1, abort_flag, p.err))) break;
@@ -385,6 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             int stV;
             if (!(ok = wait_slot(stV))) break;
+            clear_v_tail(stV, j, it.skv);
 #pragma unroll
             for (int i = 0; i < NQ; ++i) {
               if (!active(it, i, j)) continue;
@@ -417,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int r = 0; r < n_rounds && ok; ++r) {
           const int k = item_index(p, r);
           if (k < 0) continue;
-          const Item it = make_item(p, k);
+          const Item it = make_item<PAGED>(p, k);
           if (it.hi_all <= it.lo_all) continue;
           const int qb = qn % QBUF;
           if (!(ok = mbar_wait(&q_full[qb], (qn / QBUF) & 1, abort_flag, p.err))) break;
@@ -435,6 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = it.lo_all; j < it.hi_all && ok; ++j) {
             int stV;
             if (!(ok = wait_slot(stV))) break;
+            clear_v_tail(stV, j, it.skv);
             const bool next = j + 1 < it.hi_all;
             int stK1 = -1;
 #pragma unroll
@@ -489,7 +520,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int rr = 0; rr < n_rounds && ok; ++rr) {
       const int k = item_index(p, rr);
       if (k < 0) continue;
-      const Item it = make_item(p, k);
+      const Item it = make_item<PAGED>(p, k);
       const int my_lo = (i == 0) ? it.lo[0] : it.lo[1];
       const int my_hi = (i == 0) ? it.hi[0] : it.hi[1];
       const int r0 = it.q_row0 + BM * i;
@@ -700,10 +731,10 @@ int sm_count() {
   return cache[dev];
 }
 
-template <int D>
+template <int D, bool PAGED>
 cudaError_t launch_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const Params& p,
                      cudaStream_t stream) {
-  auto kern = prefill_tc_kernel<D>;
+  auto kern = prefill_tc_kernel<D, PAGED>;
   const size_t smem = Cfg<D>::SMEM;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -744,7 +775,7 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, void*
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
   p.err = err;
-  return D == 64 ? launch_d<64>(mq, mk, mv, p, stream) : launch_d<128>(mq, mk, mv, p, stream);
+  return D == 64 ? launch_d<64, false>(mq, mk, mv, p, stream) : launch_d<128, false>(mq, mk, mv, p, stream);
 }
 
 cudaError_t launch_prefill_tc_paged(const void* q, const void* k_pool, const void* v_pool, const int32_t* page_table,
@@ -774,12 +805,11 @@ cudaError_t launch_prefill_tc_paged(const void* q, const void* k_pool, const voi
   p.err = err;
   p.page_table = page_table;
   p.seq_lens = seq_lens;
-  p.paged = 1;
   p.page_size = page_size;
   p.box_rows = box_rows;
   p.max_pages = max_pages;
   p.num_pages = num_pages;
-  return D == 64 ? launch_d<64>(mq, mk, mv, p, stream) : launch_d<128>(mq, mk, mv, p, stream);
+  return D == 64 ? launch_d<64, true>(mq, mk, mv, p, stream) : launch_d<128, true>(mq, mk, mv, p, stream);
 }
 
 }  // namespace attn

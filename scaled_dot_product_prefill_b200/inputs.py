@@ -83,7 +83,6 @@ class PagedInputs:
 
 def paged_inputs(N, Hq, Hkv, D, page_size: int, seed: int, *, seq_lens=None,
                  len_range=(512, 8192), spare_pages: int = 0, poison: bool = False,
-                 tail_value: float | None = None,
                  max_pages: int | None = None, dtype: str = "bf16") -> PagedInputs:
     """A shared page pool with per-sequence page tables.
 
@@ -92,9 +91,7 @@ def paged_inputs(N, Hq, Hkv, D, page_size: int, seed: int, *, seq_lens=None,
     (plus ``spare_pages`` unreferenced ones) are scattered over the pool by
     a seeded random permutation.  With ``poison`` the unreferenced pages and
     the slots past each sequence's last token are filled with NaN, so that a
-    kernel that reads outside the valid tokens shows up as NaN output; with
-    ``tail_value`` the slots past the last token get that (finite) value
-    instead, and only the unreferenced pages get NaN.
+    kernel that lets them reach an output shows up as NaN there.
     """
     base = int(seed) * 16
     if seq_lens is None:
@@ -128,20 +125,8 @@ def paged_inputs(N, Hq, Hkv, D, page_size: int, seed: int, *, seq_lens=None,
                 phys = int(table[b, p])
                 n_tok = min(page_size, L - p * page_size)
                 valid[phys, :n_tok] = True
-        owned = torch.zeros(total, dtype=torch.bool)
-        for b, npg in enumerate(n_pages_seq):
-            owned[table[b, :npg].long()] = True
         bad = ~valid  # [total, page_size]
-        if tail_value is None:
-            k_pool = k_pool.masked_fill(bad[:, None, :, None].expand(total, Hkv, page_size, D), nan)
-            v_pool = v_pool.masked_fill(bad[:, None, :, None].expand(total, Hkv, page_size, D), nan)
-        else:
-            tail = (bad & owned[:, None])[:, None, :, None].expand(total, Hkv, page_size, D)
-            spare = (~owned)[:, None, None, None].expand(total, Hkv, page_size, D)
-            sign = torch.where(torch.arange(D) % 2 == 0, 1.0, -1.0)
-            k_pool = k_pool.masked_fill(spare, nan)
-            v_pool = v_pool.masked_fill(spare, nan)
-            k_pool = torch.where(tail, (tail_value * sign).to(k_pool.dtype), k_pool)
-            v_pool = torch.where(tail, (tail_value * sign).to(v_pool.dtype), v_pool)
+        k_pool = k_pool.masked_fill(bad[:, None, :, None].expand(total, Hkv, page_size, D), nan)
+        v_pool = v_pool.masked_fill(bad[:, None, :, None].expand(total, Hkv, page_size, D), nan)
     return PagedInputs(q, k_pool.contiguous(), v_pool.contiguous(), table,
                        seq_lens.to(torch.int32), page_size, used, seed)

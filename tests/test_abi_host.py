@@ -149,3 +149,21 @@ def test_paged_prefill_argument_validation():
     assert call(page=48) == 2
     assert call(D=96) == 2
     assert call(causal=0, window=16) == 2
+
+
+def test_kv_append_argument_validation():
+    lib = _lib()
+
+    def call(kn=FAKE, kp=FAKE, pt=FAKE, sl=FAKE, page=16, B=2, Hkv=2, S=4, D=128, num_pages=8, max_pages=4):
+        return lib.attn_kv_append(kn, FAKE, kp, FAKE, pt, sl, page, B, Hkv, S, D, num_pages, max_pages, None)
+    assert call(kn=None) == 1
+    assert call(kp=MISALIGNED) == 1
+    assert call(sl=ctypes.c_void_p(0x10002)) == 1
+    assert call(num_pages=0) == 1
+    assert call(S=-1) == 1
+    assert call(D=100) == 2              # rows must be whole 16-byte pieces
+    assert call(page=12) == 2
+    assert call(D=1024) == 2
+    assert call(kn=None, kp=None, pt=None, sl=None, B=0) == 0      # nothing to append
+    assert call(kn=None, kp=None, pt=None, sl=None, S=0) == 0
+    assert lib.attn_status_string(7) == b"ATTN_ERR_OUT_OF_PAGES"

@@ -32,6 +32,7 @@ CASES = [
     (3, 8, 1, 130, 128, 64, [40, 130, 513], True, 0),      # a cache shorter than the chunk
     (2, 8, 2, 300, 64, 128, [300, 1500], True, 200),       # sliding window
     (2, 4, 2, 200, 128, 256, [600, 201], False, 0),        # non-causal over the whole cache
+    (2, 4, 2, 100, 64, 256, [129, 250], True, 0),          # 127 and 6 NaN slots in the last 128-row box
     (1, 2, 2, 64, 64, 16, [0], True, 0),                   # an empty cache
 ]
 
@@ -39,9 +40,8 @@ CASES = [
 @pytest.mark.parametrize("case", CASES, ids=[str(c[:6]) for c in CASES])
 def test_paged_prefill_matches_oracle(case):
     B, Hq, Hkv, Sq, D, page, lens, causal, window = case
-    # unreferenced pages hold NaN (never read); slots past each last token hold large finite garbage
-    p = inputs.paged_inputs(B, Hq, Hkv, D, page, seed=sum(lens) + D, seq_lens=lens, spare_pages=3, poison=True,
-                            tail_value=3.0e4)
+    # unreferenced pages and the slots past each last token hold NaN: none may reach the output
+    p = inputs.paged_inputs(B, Hq, Hkv, D, page, seed=sum(lens) + D, seq_lens=lens, spare_pages=3, poison=True)
     q = inputs.normal((B, Hq, Sq, D), seed=99 + B)
     dev = [t.cuda() for t in (p.k_pool, p.v_pool, p.page_table, p.seq_lens)]
     out, lse = api.attn_prefill_paged(q.cuda(), *dev, max_seq_len=max(max(lens), 1), causal=causal,
@@ -85,3 +85,23 @@ def test_paged_prefill_reports_a_bad_page_without_reading_it():
     assert api.attn_device_status(clear=True) == 5      # ATTN_ERR_BAD_PAGE
     ref, _ = oracle_paged_prefill(q, p, 1 / 8.0, True, 0)
     assert_parity(out[1:], ref[1:], "bf16", "untouched sequence")
+
+
+def test_paged_prefill_never_reads_entries_past_the_last_page():
+    """Table entries after a sequence's last page hold junk (ids out of the pool, or NaN pages): no error, no NaN."""
+    lens = [201, 37, 300]
+    p = inputs.paged_inputs(3, 4, 2, 128, 16, seed=41, seq_lens=lens, spare_pages=4, poison=True, max_pages=40)
+    table = p.page_table.clone()
+    spare = sorted(set(range(p.num_pages)) - set(table[table >= 0].tolist()))
+    for b, L in enumerate(lens):
+        used = (L + 15) // 16
+        table[b, used::2] = 1 << 30
+        table[b, used + 1::2] = spare[b % len(spare)]
+    q = inputs.normal((3, 4, 64, 128), seed=42)
+    api.attn_device_status(clear=True)
+    out = api.attn_prefill_paged(q.cuda(), p.k_pool.cuda(), p.v_pool.cuda(), table.cuda(), p.seq_lens.cuda(),
+                                 max_seq_len=300, causal=False)
+    torch.cuda.synchronize()
+    assert api.attn_device_status(clear=True) == 0
+    ref, _ = oracle_paged_prefill(q, p, 1 / np.sqrt(128), False, 0)
+    assert_parity(out, ref, "bf16", "junk past the last page")

@@ -14,6 +14,7 @@ from oracle import sdpa
 _orig_visible = sdpa.visible
 _orig_softmax = sdpa.softmax_rows
 _orig_weights = sdpa.weights
+_orig_append = sdpa.append_pages
 
 
 def _visible_window_off_by_one(Sq, Skv, causal, window=0, rows=None):
@@ -55,6 +56,14 @@ def _weights_keys_reversed(q, k, scale, causal, window=0, rows=None, Sq=None):
     return P[:, ::-1], lse
 
 
+def _append_one_slot_late(pool, page_table, seq_lens, new, page_size):
+    return _orig_append(pool, page_table, [int(L) + 1 for L in seq_lens], new, page_size)
+
+
+def _append_chunk_reversed(pool, page_table, seq_lens, new, page_size):
+    return _orig_append(pool, page_table, seq_lens, np.asarray(new)[:, :, ::-1], page_size)
+
+
 MUTATIONS = {
     "kv_head round robin": ("kv_head", lambda h, Hq, Hkv: h % Hkv),
     "window off by one": ("visible", _visible_window_off_by_one),
@@ -64,6 +73,8 @@ MUTATIONS = {
     "mask after softmax": ("weights", _weights_mask_after_softmax),
     "scale squared": ("weights", _weights_scale_by_d),
     "value rows reversed": ("weights", _weights_keys_reversed),
+    "append one slot late": ("append_pages", _append_one_slot_late),
+    "append chunk reversed": ("append_pages", _append_chunk_reversed),
 }
 
 PIN_TESTS = [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]

@@ -330,3 +330,63 @@ def test_lse_matches_python_log_sum_exp_and_merges_disjoint_key_sets():
     w1, w2 = np.exp(l1 - lf)[..., None], np.exp(l2 - lf)[..., None]
     np.testing.assert_allclose(w1 * o1 + w2 * o2, full, atol=1e-13)
     np.testing.assert_allclose(np.logaddexp(l1, l2), lf, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# appending to the paged cache
+
+
+def _random_table(rng, B, max_pages, num_pages):
+    perm = rng.permutation(num_pages)[:B * max_pages]
+    return perm.reshape(B, max_pages).astype(np.int64)
+
+
+def test_append_then_gather_returns_the_appended_tokens():
+    """Chunks appended one after another read back, through the page table, as their concatenation."""
+    rng = np.random.default_rng(7)
+    B, Hkv, D, page = 3, 2, 4, 4
+    table = _random_table(rng, B, 6, 30)           # non-contiguous, shuffled pages
+    pool = np.full((30, Hkv, page, D), np.nan)
+    written = [[] for _ in range(B)]
+    lens = np.zeros(B, dtype=np.int64)
+    for S_new in (5, 1, 1, 3, 7):                  # a prefill chunk, decode steps, more chunks
+        new = rng.standard_normal((B, Hkv, S_new, D))
+        lens = lens + S_new
+        pool = sdpa.append_pages(pool, table, lens, new, page)
+        for b in range(B):
+            written[b].append(new[b].transpose(1, 0, 2))        # [S_new, Hkv, D]
+    for b in range(B):
+        want = np.concatenate(written[b])
+        got = sdpa.gather_pages(pool, table[b], int(lens[b]), page)
+        np.testing.assert_array_equal(got, want)
+    # nothing else was written: exactly the appended slots lost their NaN
+    assert np.count_nonzero(~np.isnan(pool)) == int(lens.sum()) * Hkv * D
+
+
+def test_append_of_a_chunk_longer_than_the_cache_keeps_only_its_last_tokens():
+    B, Hkv, D, page = 2, 1, 2, 4
+    table = np.array([[3, 1], [0, 2]])
+    pool = np.full((4, Hkv, page, D), np.nan)
+    new = np.arange(B * Hkv * 5 * D, dtype=np.float64).reshape(B, Hkv, 5, D)
+    out = sdpa.append_pages(pool, table, [2, 5], new, page)
+    # sequence 0 holds 2 tokens: the chunk's tokens 3 and 4 at positions 0 and 1
+    np.testing.assert_array_equal(out[3, 0, :2], new[0, 0, 3:])
+    assert np.isnan(out[3, 0, 2:]).all() and np.isnan(out[1]).all()
+    np.testing.assert_array_equal(sdpa.gather_pages(out, table[1], 5, page), new[1].transpose(1, 0, 2))
+
+
+def test_append_then_decode_equals_full_causal_recompute():
+    """Prefill a prompt into the cache, then decode token by token: each step equals the causal row."""
+    S, P, H, D, page = 11, 4, 2, 8, 4
+    q, k, v = rand(1, H, S, D), rand(1, H, S, D), rand(1, H, S, D)
+    full = sdpa.attention(q, k, v, 0.3, causal=True)
+    table = np.array([[5, 0, 3]])
+    k_pool = np.full((6, H, page, D), np.nan)
+    v_pool = np.full((6, H, page, D), np.nan)
+    k_pool = sdpa.append_pages(k_pool, table, [P], k[:, :, :P], page)
+    v_pool = sdpa.append_pages(v_pool, table, [P], v[:, :, :P], page)
+    for t in range(P, S):
+        k_pool = sdpa.append_pages(k_pool, table, [t + 1], k[:, :, t:t + 1], page)
+        v_pool = sdpa.append_pages(v_pool, table, [t + 1], v[:, :, t:t + 1], page)
+        step = sdpa.decode_paged(q[0, :, t][None], k_pool, v_pool, table, [t + 1], page, 0.3)
+        np.testing.assert_allclose(step[0], full[0, :, t], atol=1e-14)
