@@ -24,8 +24,12 @@ LIB = os.path.join(PKG, "libattn_b200.so")
 
 SOURCES = ["attn_api.cu", "prefill_sm100.cu", "prefill_f32.cu", "decode_paged.cu", "kv_append.cu", "page_pool.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
-         "-I", INCLUDE, "-I", CSRC]
+# Host code is built without exceptions and uses only the C library and
+# pthreads, so the .so needs no C++ runtime: a late dlopen of libstdc++ can
+# fail for want of static TLS when the host process has not loaded it yet.
+FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fno-exceptions",
+         "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]
+LINK_FLAGS = ["-Xlinker", "--as-needed", "-lpthread"]
 
 
 def nvcc() -> str:
@@ -74,7 +78,7 @@ def build(verbose: bool = False, extra=()) -> str:
                 print(msg)
     objs = [o for o, _ in results]
     if _stale(LIB, objs) or extra:
-        cmd = [nvcc()] + ARCH + ["-shared", "-o", LIB] + objs
+        cmd = [nvcc()] + ARCH + ["-shared", "-o", LIB] + objs + LINK_FLAGS
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed: {' '.join(cmd)}\n{r.stdout}\n{r.stderr}")

@@ -5,7 +5,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cuda_runtime.h>
-#include <mutex>
+#include <pthread.h>
 
 #include "attn_b200.h"
 #include "common.cuh"
@@ -18,16 +18,17 @@ __device__ unsigned int g_error_word = 0;
 unsigned int* device_error_word() {
   constexpr int kMaxDevices = 64;
   static unsigned int* addr[kMaxDevices] = {};
-  static std::mutex mu;
+  static pthread_mutex_t mu = PTHREAD_MUTEX_INITIALIZER;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
+  pthread_mutex_lock(&mu);
   if (addr[dev] == nullptr) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
-    addr[dev] = static_cast<unsigned int*>(p);
+    if (cudaGetSymbolAddress(&p, g_error_word) == cudaSuccess) addr[dev] = static_cast<unsigned int*>(p);
   }
-  return addr[dev];
+  unsigned int* a = addr[dev];
+  pthread_mutex_unlock(&mu);
+  return a;
 }
 
 }  // namespace attn

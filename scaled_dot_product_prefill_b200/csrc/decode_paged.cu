@@ -32,7 +32,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cuda_bf16.h>
-#include <mutex>
+#include <pthread.h>
 
 #include "common.cuh"
 #include "sm100_ptx.cuh"
@@ -530,16 +530,17 @@ size_t decode_scratch_capacity() { return kDecodeScratchBytes; }
 void* decode_scratch_address() {
   constexpr int kMaxDevices = 64;
   static void* addr[kMaxDevices] = {};
-  static std::mutex mu;
+  static pthread_mutex_t mu = PTHREAD_MUTEX_INITIALIZER;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
+  pthread_mutex_lock(&mu);
   if (addr[dev] == nullptr) {
     void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess) return nullptr;
-    addr[dev] = ptr;
+    if (cudaGetSymbolAddress(&ptr, g_decode_scratch) == cudaSuccess) addr[dev] = ptr;
   }
-  return addr[dev];
+  void* a = addr[dev];
+  pthread_mutex_unlock(&mu);
+  return a;
 }
 
 }  // namespace attn

@@ -37,7 +37,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
-#include <mutex>
+#include <pthread.h>
 
 #include "common.cuh"
 #include "sm100_ptx.cuh"
@@ -56,8 +56,8 @@ constexpr int kMmaWarp = 9;
 // and MMA warps, two idle warps) gets kProducerRegs.  The split must fit the
 // launch allocation: 128 * (2 * kSoftmaxRegs + kProducerRegs) <= kThreads *
 // regs-per-thread at launch, which the host checks before every launch.
-constexpr int kSoftmaxRegs = 200;
-constexpr int kProducerRegs = 104;
+constexpr int kSoftmaxRegs = 208;
+constexpr int kProducerRegs = 88;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kTau = 8.0f;     // lazy-rescale threshold, log2 units
 // Of every 16 score pairs of a row, how many take exp2 on the FMA pipe
@@ -515,6 +515,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
     int t = 0, oc = 0;
     int pv = 0;   // SEP_P: P_i V products of this tile completed and waited for
+    // O_i *= alpha (every row of the warp takes part when any row needs it)
+    auto rescale_o = [&](bool later_tile, float alpha) {
+      if (!__any_sync(0xffffffffu, later_tile && alpha != 1.f)) return;
+      const uint64_t a2 = f2_pack(alpha, alpha);
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(o_tmem + 32 * c, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float x0, x1;
+          f2_unpack(f2_mul(f2_pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2), x0, x1);
+          o[e] = __float_as_uint(x0);
+          o[e + 1] = __float_as_uint(x1);
+        }
+        tmem_st32(o_tmem + 32 * c, o);
+      }
+    };
     bool ok = true;
 
     for (int rr = 0; rr < n_rounds && ok; ++rr) {
@@ -576,36 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           l *= alpha;
           m_ref = m_tile;
         }
-        if constexpr (C::SEP_P) {
-          // P_i(j-1) V must be complete before O_i is rescaled or P_i rewritten
-          if (j > my_lo) {
-            ok = mbar_wait(&o_done[i], pv & 1, abort_flag, p.err);
-            ++pv;
-            if (!__all_sync(0xffffffffu, ok)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-          }
-        }
-        const bool rescale = (j > my_lo) && (alpha != 1.f);
-        if (__any_sync(0xffffffffu, rescale)) {
-          const uint64_t a2 = f2_pack(alpha, alpha);
-#pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(o_tmem + 32 * c, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              float x0, x1;
-              f2_unpack(f2_mul(f2_pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2), x0, x1);
-              o[e] = __float_as_uint(x0);
-              o[e + 1] = __float_as_uint(x1);
-            }
-            tmem_st32(o_tmem + 32 * c, o);
-          }
-        }
+        if constexpr (!C::SEP_P) rescale_o(j > my_lo, alpha);   // O_i is current: S_i(j) covers P_i V(j-1)
         const float mb = (m_ref == -INFINITY) ? 0.f : m_ref;
         const uint64_t nm2 = f2_pack(-mb, -mb);
         uint32_t pk[BN / 2];
@@ -631,6 +621,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         f2_unpack(f2_add(sum2[0], sum2[1]), s0, s1);
         f2_unpack(f2_add(sum2[2], sum2[3]), s2, s3);
         l += (s0 + s1) + (s2 + s3);
+        // The exponentials above need nothing from tensor memory; only now must
+        // P_i(j-1) V be complete: before O_i is rescaled and (separate P) before
+        // P_i is rewritten.  Waiting here hides that product behind them.
+        if constexpr (C::SEP_P) {
+          if (j > my_lo) {
+            ok = mbar_wait(&o_done[i], pv & 1, abort_flag, p.err);
+            ++pv;
+            if (!__all_sync(0xffffffffu, ok)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
+        }
+        if constexpr (C::SEP_P) rescale_o(j > my_lo, alpha);
 #pragma unroll
         for (int c = 0; c < BN / 64; ++c) tmem_st32(p_tmem + 32 * c, pk + 32 * c);
         tmem_wait_st();
@@ -690,18 +695,21 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+EncodeTiledFn g_encoder = nullptr;
+
+void look_up_encoder() {
+  void* ptr = nullptr;
+  cudaDriverEntryPointQueryResult q{};
+  if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+          cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    g_encoder = reinterpret_cast<EncodeTiledFn>(ptr);
+}
+
 EncodeTiledFn tensor_map_encoder() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q{};
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  });
-  return fn;
+  static pthread_once_t once = PTHREAD_ONCE_INIT;
+  pthread_once(&once, look_up_encoder);
+  return g_encoder;
 }
 
 // [planes][rows][D] bf16 tensor, boxes of 64 columns x box_rows rows, 128-byte swizzle.

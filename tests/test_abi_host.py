@@ -167,3 +167,26 @@ def test_kv_append_argument_validation():
     assert call(kn=None, kp=None, pt=None, sl=None, B=0) == 0      # nothing to append
     assert call(kn=None, kp=None, pt=None, sl=None, S=0) == 0
     assert lib.attn_status_string(7) == b"ATTN_ERR_OUT_OF_PAGES"
+
+
+def test_library_needs_no_cxx_runtime_and_loads_first():
+    """The .so depends on the C library alone, and loads in a process that has loaded nothing else.
+
+    A C++ runtime pulled in by a late dlopen can fail for want of static TLS;
+    the library avoids needing one at all.
+    """
+    import subprocess
+    import sys
+
+    from scaled_dot_product_prefill_b200 import _lib as L
+
+    _lib()
+    path = L.lib_path()
+    with open(path, "rb") as f:
+        data = f.read()
+    for name in (b"libstdc++.so", b"libgcc_s.so"):
+        assert name not in data, f"{path} references {name.decode()}"
+    code = f"import ctypes; lib = ctypes.CDLL({path!r}); print(lib.attn_version())"
+    out = subprocess.run([sys.executable, "-S", "-c", code], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stderr
+    assert int(out.stdout.strip()) >= 100
