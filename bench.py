@@ -277,6 +277,7 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0 and not args.no_extra:
         extra = other_workloads(dev, peaks)
         extra.update(append_workloads(dev, peaks))
+        extra.update(fp8_decode_workload(dev, peaks))
 
     result = None
     if rank == 0:
@@ -377,6 +378,37 @@ def graph_prefill_ms(fn, flush, reps):
     ms = float(np.median([a.elapsed_time(b) for a, b in ev]))
     del g
     return ms
+
+
+def fp8_decode_workload(dev, peaks):
+    """attn_decode_paged_fp8 on the paged_decode_gqa shape with an E4M3 cache (1 byte per K/V element)."""
+    import torch
+
+    from scaled_dot_product_prefill_b200 import api
+
+    dspec = DECODE
+    ks = vs = 1.0 / 64
+    pd = inputs.paged_inputs_fp8(dspec.N, dspec.Hq, dspec.Hkv, dspec.D, dspec.page_size, dspec.seed, k_scale=ks,
+                                 v_scale=vs, len_range=dspec.len_range)
+    dq, kp, vp, pt, sl = (t.to(dev) for t in (pd.q, pd.k_pool, pd.v_pool, pd.page_table, pd.seq_lens))
+    out = torch.empty_like(dq)
+    msl = pd.max_seq_len
+    ws = torch.empty(api.attn_decode_paged_workspace_size(dspec.N, dspec.Hq, dspec.D, msl, dspec.page_size),
+                     dtype=torch.uint8, device=dev)
+    ms = time_call(lambda: api.attn_decode_paged_fp8(dq, kp, vp, pt, sl, max_seq_len=msl, k_scale=ks, v_scale=vs,
+                                                     scale=dspec.scale, workspace=ws, out=out), 100)
+    lens = pd.seq_lens.numpy()
+    kv = int(lens.sum()) * dspec.Hkv * dspec.D * 2          # K and V, one byte each
+    nbytes = kv + workloads.decode_bytes(lens, dspec.Hq, dspec.Hkv, dspec.D, dspec.page_size) - \
+        workloads.kv_bytes(lens, dspec.Hkv, dspec.D)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    res = {"decode_fp8_" + dspec.name: {"ms": round(ms, 5), "GB/s": round(gbs, 1), "bytes": int(nbytes),
+                                        "frac_of_hbm": round(gbs / float(peaks["hbm_gbs"]), 4),
+                                        "tokens_per_s": round(int(lens.sum()) / (ms * 1e-3), 1),
+                                        "l2": "none (0.57 GB of K/V > L2)"}}
+    del kp, vp
+    torch.cuda.empty_cache()
+    return res
 
 
 def append_workloads(dev, peaks):

@@ -250,6 +250,26 @@ attn_status_t attn_decode_paged_noalloc(const void* q, const void* k_pool, const
                                         int num_pages, int max_pages, int max_seq_len,
                                         float scale, int window, void* out, attn_stream_t stream);
 
+/*
+ * attn_decode_paged_fp8 -- attn_decode_paged over a cache stored as 8-bit
+ * floats: k_pool and v_pool hold FP8 E4M3 codes (1 sign, 4 exponent bits with
+ * bias 7, 3 mantissa bits, subnormals; no infinity; the codes 0x7F and 0xFF
+ * are NaN), one byte per element, in the same [num_pages, Hkv, page_size, D]
+ * layout.  An element stands for k_scale * e4m3(code) (v_scale for V):
+ *     O = softmax((q . k_scale*K) * scale) (v_scale*V).
+ * q and out stay bf16.  The pages give no 8-bit cache: this is a storage
+ * variant of the decode above that halves the bytes it reads, with the same
+ * arithmetic after the exact conversion of each code.
+ * k_scale, v_scale: finite and > 0.  Every other argument, the workspace
+ * (attn_decode_paged_workspace_size) and the errors are as attn_decode_paged.
+ */
+attn_status_t attn_decode_paged_fp8(const void* q, const uint8_t* k_pool, const uint8_t* v_pool,
+                                    const int32_t* page_table, const int32_t* seq_lens,
+                                    int page_size, int N, int Hq, int Hkv, int D,
+                                    int num_pages, int max_pages, int max_seq_len,
+                                    float scale, float k_scale, float v_scale, int window,
+                                    void* workspace, size_t workspace_bytes, void* out, attn_stream_t stream);
+
 /* Bytes of workspace attn_decode_paged needs for these sizes (0 if any size
  * is invalid).  Pure host arithmetic, no CUDA call. */
 size_t attn_decode_paged_workspace_size(int N, int Hq, int D, int max_seq_len, int page_size);

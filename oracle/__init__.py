@@ -36,9 +36,11 @@ Modules:
   sampled rows, paged gather and paged decode.
 * ``brute`` -- pure-Python loops with ``math.exp``: an independent second
   statement of the same definition for tiny shapes.
+* ``fp8``   -- the value of each FP8 E4M3 code, for the 8-bit paged cache
+  (decoded, then fed to ``sdpa`` like any other cache).
 
 Every function is pinned by ``tests/test_oracle_pins.py`` against closed
 forms, invariants and the values the pages print (``tests/golden/``); none
 is "parity unpinned".
 """
-from . import brute, sdpa  # noqa: F401
+from . import brute, fp8, sdpa  # noqa: F401

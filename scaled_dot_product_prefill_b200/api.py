@@ -15,7 +15,7 @@ from ._lib import AttnError
 
 __all__ = ["attn_prefill", "attn_prefill_f32", "attn_prefill_lse", "attn_prefill_f32_lse",
            "attn_prefill_paged", "attn_decode_paged", "attn_decode_paged_noalloc",
-           "attn_decode_paged_workspace_size", "attn_kv_append", "PagePool",
+           "attn_decode_paged_workspace_size", "attn_decode_paged_fp8", "attn_kv_append", "PagePool",
            "attn_device_status", "attn_status_string", "attn_version", "AttnError"]
 
 
@@ -161,6 +161,31 @@ def attn_decode_paged(q, k_pool, v_pool, page_table, seq_lens, *, max_seq_len, s
         _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(page_table), _ptr(seq_lens), page_size, N, Hq, Hkv, D,
         num_pages, max_pages, int(max_seq_len), float(scale), int(window), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(out), _stream(stream)))
+    return out
+
+
+def attn_decode_paged_fp8(q, k_pool, v_pool, page_table, seq_lens, *, max_seq_len, k_scale, v_scale, scale=None,
+                          window=0, workspace=None, out=None, stream=None):
+    """Paged decode over an 8-bit cache: pools are uint8 E4M3 codes [P,Hkv,page,D]; element = scale * e4m3(code)."""
+    N, Hq, D = q.shape
+    num_pages, Hkv, page_size, _ = k_pool.shape
+    max_pages = page_table.shape[1]
+    if k_pool.dtype != torch.uint8 or v_pool.dtype != torch.uint8:
+        raise ValueError("k_pool and v_pool must hold uint8 E4M3 codes")
+    if out is None:
+        out = torch.empty_like(q)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    need = attn_decode_paged_workspace_size(N, Hq, D, max_seq_len, page_size)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _need_cuda(q, k_pool, v_pool, page_table, seq_lens, out, workspace)
+    if page_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise ValueError("page_table and seq_lens must be int32")
+    _check("attn_decode_paged_fp8", _lib.load().attn_decode_paged_fp8(
+        _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(page_table), _ptr(seq_lens), page_size, N, Hq, Hkv, D,
+        num_pages, max_pages, int(max_seq_len), float(scale), float(k_scale), float(v_scale), int(window),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(out), _stream(stream)))
     return out
 
 

@@ -195,14 +195,21 @@ size_t attn_decode_paged_workspace_size(int N, int Hq, int D, int max_seq_len, i
   return attn::decode_workspace_bytes(N, Hq, D, max_seq_len, page_size);
 }
 
-attn_status_t attn_decode_paged(const void* q, const void* k_pool, const void* v_pool, const int32_t* page_table,
-                                const int32_t* seq_lens, int page_size, int N, int Hq, int Hkv, int D,
-                                int num_pages, int max_pages, int max_seq_len, float scale, int window,
-                                void* workspace, size_t workspace_bytes, void* out, attn_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+attn_status_t decode_paged(const void* q, const void* k_pool, const void* v_pool, const int32_t* page_table,
+                           const int32_t* seq_lens, int page_size, int N, int Hq, int Hkv, int D, int num_pages,
+                           int max_pages, int max_seq_len, float scale, int window, void* workspace,
+                           size_t workspace_bytes, void* out, attn_stream_t stream, bool fp8, float k_scale,
+                           float v_scale) {
   if (N < 0 || Hq < 0 || Hkv < 0 || D <= 0 || num_pages < 0 || max_pages < 0 || max_seq_len < 0 || window < 0 ||
       page_size <= 0)
     return ATTN_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (!(k_scale > 0.f) || !std::isfinite(k_scale) || !(v_scale > 0.f) || !std::isfinite(v_scale))
+    return ATTN_ERR_INVALID_ARG;
   if (N == 0 || Hq == 0) return ATTN_OK;
   if (Hkv == 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
   if (q == nullptr || out == nullptr || seq_lens == nullptr) return ATTN_ERR_INVALID_ARG;
@@ -220,7 +227,29 @@ attn_status_t attn_decode_paged(const void* q, const void* k_pool, const void* v
   if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)) return ATTN_ERR_WORKSPACE;
   return from_cuda(attn::launch_decode_paged(q, k_pool, v_pool, page_table, seq_lens, page_size, N, Hq, Hkv, D,
                                              num_pages, max_pages, max_seq_len, scale, window, workspace, out,
-                                             attn::device_error_word(), reinterpret_cast<cudaStream_t>(stream)));
+                                             attn::device_error_word(), reinterpret_cast<cudaStream_t>(stream), fp8,
+                                             k_scale, v_scale));
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status_t attn_decode_paged(const void* q, const void* k_pool, const void* v_pool, const int32_t* page_table,
+                                const int32_t* seq_lens, int page_size, int N, int Hq, int Hkv, int D,
+                                int num_pages, int max_pages, int max_seq_len, float scale, int window,
+                                void* workspace, size_t workspace_bytes, void* out, attn_stream_t stream) {
+  return decode_paged(q, k_pool, v_pool, page_table, seq_lens, page_size, N, Hq, Hkv, D, num_pages, max_pages,
+                      max_seq_len, scale, window, workspace, workspace_bytes, out, stream, false, 1.f, 1.f);
+}
+
+attn_status_t attn_decode_paged_fp8(const void* q, const uint8_t* k_pool, const uint8_t* v_pool,
+                                    const int32_t* page_table, const int32_t* seq_lens, int page_size, int N, int Hq,
+                                    int Hkv, int D, int num_pages, int max_pages, int max_seq_len, float scale,
+                                    float k_scale, float v_scale, int window, void* workspace,
+                                    size_t workspace_bytes, void* out, attn_stream_t stream) {
+  return decode_paged(q, k_pool, v_pool, page_table, seq_lens, page_size, N, Hq, Hkv, D, num_pages, max_pages,
+                      max_seq_len, scale, window, workspace, workspace_bytes, out, stream, true, k_scale, v_scale);
 }
 
 attn_status_t attn_decode_paged_noalloc(const void* q, const void* k_pool, const void* v_pool,

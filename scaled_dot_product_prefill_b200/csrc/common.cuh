@@ -51,7 +51,8 @@ void* decode_scratch_address();
 cudaError_t launch_decode_paged(const void* q, const void* k_pool, const void* v_pool, const int32_t* page_table,
                                 const int32_t* seq_lens, int page_size, int N, int Hq, int Hkv, int D,
                                 int num_pages, int max_pages, int max_seq_len, float scale, int window,
-                                void* workspace, void* out, unsigned int* err, cudaStream_t stream);
+                                void* workspace, void* out, unsigned int* err, cudaStream_t stream,
+                                bool fp8 = false, float k_scale = 1.f, float v_scale = 1.f);
 
 // k_new/v_new [B, Hkv, S_new, D] -> pools [num_pages, Hkv, page_size, D] at positions seq_lens[b] - S_new + i.
 cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* k_pool, void* v_pool,

@@ -57,8 +57,8 @@ constexpr float kTau = 8.0f;    // lazy-rescale threshold, log2 units
 
 struct DecodeParams {
   const __nv_bfloat16* q;
-  const __nv_bfloat16* k_pool;
-  const __nv_bfloat16* v_pool;
+  const void* k_pool;   // bf16 or fp8 e4m3 codes, [num_pages, Hkv, page_size, D]
+  const void* v_pool;
   const int32_t* page_table;
   const int32_t* seq_lens;
   float* ws_o;        // [N, Hq, max_splits, D]
@@ -67,7 +67,8 @@ struct DecodeParams {
   unsigned int* err;
   int page_size, Hq, Hkv, num_pages, max_pages, max_seq_len;
   int split_tokens, max_splits, window;
-  float scale_log2;
+  float scale_log2;   // softmax scale (times the K scale for fp8) in log2 units
+  float v_scale;      // output multiplier: the V scale for fp8, 1 for bf16
 };
 
 // 8 bf16 (one 16-byte load) as 4 packed fp32 pairs (element 2i in the low half).
@@ -75,6 +76,40 @@ __device__ __forceinline__ void bf16x8_to_f2(const uint4& u, uint64_t (&f)[4]) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) f[i] = f2_pack(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+}
+
+// 8 fp8 e4m3 codes (one 8-byte load) as 4 packed fp32 pairs (element 2i in the
+// low half): the hardware conversion to f16 pairs is exact, as is f16 -> f32.
+__device__ __forceinline__ void fp8x8_to_f2(const uint2& u, uint64_t (&f)[4]) {
+  const uint32_t w[2] = {u.x, u.y};
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const unsigned short pair = static_cast<unsigned short>(w[i] >> (16 * h));
+      uint32_t h2;
+      asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(pair));
+      float lo, hi;
+      asm("{\n\t.reg .f16 l, u;\n\tmov.b32 {l, u}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, u;\n\t}"
+          : "=f"(lo), "=f"(hi)
+          : "r"(h2));
+      f[2 * i + h] = f2_pack(lo, hi);
+    }
+  }
+}
+
+// One lane's 8 elements of a K or V row from shared memory as packed fp32 pairs.
+template <bool FP8>
+__device__ __forceinline__ void load8_f2(const uint8_t* base, int idx, bool zero, uint64_t (&f)[4]) {
+  if constexpr (FP8) {
+    uint2 u = reinterpret_cast<const uint2*>(base)[idx];
+    if (zero) u = make_uint2(0u, 0u);
+    fp8x8_to_f2(u, f);
+  } else {
+    uint4 u = reinterpret_cast<const uint4*>(base)[idx];
+    if (zero) u = make_uint4(0u, 0u, 0u, 0u);
+    bf16x8_to_f2(u, f);
+  }
 }
 
 // Sum NV per-lane values over groups of R lanes (lane bits below R) and
@@ -105,34 +140,40 @@ __device__ __forceinline__ void reduce_scatter(float (&v)[NV], int lane, int& ba
   }
 }
 
-template <int D>
+// FP8: K and V are e4m3 codes (1 byte per element) instead of bf16.  Every lane
+// handles 8 elements of a row either way, so the ring keeps its bytes and
+// holds twice the chunks for fp8.
+template <int D, bool FP8>
 struct Geo {
-  static constexpr int R = D / 8;                 // lanes per token row (16 B each)
-  static constexpr int TPL = 32 / R;              // tokens per warp-wide 16 B load
+  static constexpr int EB = FP8 ? 1 : 2;          // bytes per element
+  static constexpr int R = D / 8;                 // lanes per token row (8 elements each)
+  static constexpr int TPL = 32 / R;              // tokens per warp-wide load
   static constexpr int NL = kChunk / TPL;         // loads per chunk per lane
-  static constexpr int CHUNK_BYTES = kChunk * D * 2;
-  static constexpr int STAGES = (D == 128) ? ATTN_DECODE_STAGES : 2 * ATTN_DECODE_STAGES;
+  static constexpr int CHUNK_BYTES = kChunk * D * EB;
+  static constexpr int STAGES = ((D == 128) ? ATTN_DECODE_STAGES : 2 * ATTN_DECODE_STAGES) * (FP8 ? 2 : 1);
 };
 
-template <int D, int G>
+template <int D, int G, bool FP8>
 struct SplitSmem {
-  alignas(1024) uint8_t ring[kWarps][Geo<D>::STAGES][2][Geo<D>::CHUNK_BYTES];  // K then V
+  alignas(1024) uint8_t ring[kWarps][Geo<D, FP8>::STAGES][2][Geo<D, FP8>::CHUNK_BYTES];  // K then V
   alignas(16) float pbuf[kWarps][kChunk * G];     // p of the current chunk, [token][head]
   float wm[kWarps][G];                            // per-warp reference max (log2 units)
   float wl[kWarps][G];                            // per-warp running sum
-  uint64_t full[kWarps][Geo<D>::STAGES];
-  int stage_ok[kWarps][Geo<D>::STAGES];
+  uint64_t full[kWarps][Geo<D, FP8>::STAGES];
+  int stage_ok[kWarps][Geo<D, FP8>::STAGES];
 };
 
-template <int D, int G>
-__global__ void __launch_bounds__(kWarps * 32, ATTN_DECODE_MINB) decode_split_kernel(const DecodeParams p) {
-  using Gm = Geo<D>;
+// Groups of 8 query heads hold twice the accumulators: 2 CTAs per SM leave them 255 registers.
+template <int D, int G, bool FP8>
+__global__ void __launch_bounds__(kWarps * 32, (G >= 8) ? 2 : ATTN_DECODE_MINB)
+    decode_split_kernel(const DecodeParams p) {
+  using Gm = Geo<D, FP8>;
   constexpr int R = Gm::R, TPL = Gm::TPL, NL = Gm::NL, STAGES = Gm::STAGES;
   constexpr int NV = NL * G;                       // partial dot products per lane per chunk
   constexpr int NF = (NV / R) > 0 ? (NV / R) : 1;  // scores held per lane after reduction
   constexpr int DUP = (NV >= R) ? 1 : R / NV;       // lanes sharing one score when NV < R
   extern __shared__ uint8_t smem_raw[];
-  SplitSmem<D, G>& sm = *reinterpret_cast<SplitSmem<D, G>*>(
+  SplitSmem<D, G, FP8>& sm = *reinterpret_cast<SplitSmem<D, G, FP8>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
 
   const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
@@ -183,8 +224,8 @@ __global__ void __launch_bounds__(kWarps * 32, ATTN_DECODE_MINB) decode_split_ke
         const size_t off = (static_cast<size_t>(phys) * p.Hkv + g) * head_stride +
                            static_cast<size_t>(t0 % p.page_size) * D;
         mbar_arrive_expect_tx(bar, 2 * Gm::CHUNK_BYTES);
-        bulk_load(sm.ring[warp][st][0], p.k_pool + off, Gm::CHUNK_BYTES, bar);
-        bulk_load(sm.ring[warp][st][1], p.v_pool + off, Gm::CHUNK_BYTES, bar);
+        bulk_load(sm.ring[warp][st][0], static_cast<const uint8_t*>(p.k_pool) + off * Gm::EB, Gm::CHUNK_BYTES, bar);
+        bulk_load(sm.ring[warp][st][1], static_cast<const uint8_t*>(p.v_pool) + off * Gm::EB, Gm::CHUNK_BYTES, bar);
       }
     }
   };
@@ -229,15 +270,15 @@ __global__ void __launch_bounds__(kWarps * 32, ATTN_DECODE_MINB) decode_split_ke
     const int chunk_t0 = (c_begin + warp + kWarps * i) * kChunk;
     const bool stage_ok = sm.stage_ok[warp][st] != 0;
     const bool full = stage_ok && chunk_t0 >= lo && chunk_t0 + kChunk <= L;
-    const uint4* sk = reinterpret_cast<const uint4*>(sm.ring[warp][st][0]);
-    const uint4* sv = reinterpret_cast<const uint4*>(sm.ring[warp][st][1]);
+    const uint8_t* sk = sm.ring[warp][st][0];
+    const uint8_t* sv = sm.ring[warp][st][1];
 
     // ---- scores: partial dot products over my 8 columns, then reduce over the row's R lanes
     float part[NV];
 #pragma unroll
     for (int l = 0; l < NL; ++l) {
       uint64_t k2[4];
-      bf16x8_to_f2(sk[l * 32 + lane], k2);
+      load8_f2<FP8>(sk, l * 32 + lane, false, k2);
 #pragma unroll
       for (int hh = 0; hh < G; ++hh) {
         uint64_t a = f2_mul(q2[hh][0], k2[0]);
@@ -308,13 +349,13 @@ __global__ void __launch_bounds__(kWarps * 32, ATTN_DECODE_MINB) decode_split_ke
 #pragma unroll
     for (int l = 0; l < NL; ++l) {
       const int tok = l * TPL + lane / R;
-      uint4 u = sv[l * 32 + lane];
+      bool zero = false;
       if (!full) {
         const int t = chunk_t0 + tok;
-        if (!(stage_ok && t >= lo && t < L)) u = make_uint4(0u, 0u, 0u, 0u);  // poisoned slots stay out
+        zero = !(stage_ok && t >= lo && t < L);   // poisoned slots stay out
       }
       uint64_t v2[4];
-      bf16x8_to_f2(u, v2);
+      load8_f2<FP8>(sv, l * 32 + lane, zero, v2);
 #pragma unroll
       for (int hh = 0; hh < G; ++hh) {
         const float pr = pb[tok * G + hh];
@@ -417,7 +458,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
       }
     }
   }
-  const float inv = (wsum > 0.f) ? 1.f / wsum : 0.f;
+  const float inv = (wsum > 0.f) ? p.v_scale / wsum : 0.f;
 #pragma unroll
   for (int t = 0; t < PER; t += 2) {
     __nv_bfloat162 v2 = __floats2bfloat162_rn(acc[t] * inv, acc[t + 1] * inv);
@@ -425,10 +466,10 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
   }
 }
 
-template <int D, int G>
+template <int D, int G, bool FP8>
 cudaError_t launch_split(const DecodeParams& p, int N, cudaStream_t stream) {
-  const size_t smem = sizeof(SplitSmem<D, G>) + 1024;
-  auto kern = decode_split_kernel<D, G>;
+  const size_t smem = sizeof(SplitSmem<D, G, FP8>) + 1024;
+  auto kern = decode_split_kernel<D, G, FP8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(p.max_splits, p.Hkv, N);
@@ -465,12 +506,13 @@ size_t decode_workspace_bytes(int N, int Hq, int D, int max_seq_len, int page_si
 cudaError_t launch_decode_paged(const void* q, const void* k_pool, const void* v_pool, const int32_t* page_table,
                                 const int32_t* seq_lens, int page_size, int N, int Hq, int Hkv, int D,
                                 int num_pages, int max_pages, int max_seq_len, float scale, int window,
-                                void* workspace, void* out, unsigned int* err, cudaStream_t stream) {
+                                void* workspace, void* out, unsigned int* err, cudaStream_t stream, bool fp8,
+                                float k_scale, float v_scale) {
   const DecodeGeometry geo = decode_geometry(N, Hq, D, max_seq_len, page_size);
   DecodeParams p{};
   p.q = static_cast<const __nv_bfloat16*>(q);
-  p.k_pool = static_cast<const __nv_bfloat16*>(k_pool);
-  p.v_pool = static_cast<const __nv_bfloat16*>(v_pool);
+  p.k_pool = k_pool;
+  p.v_pool = v_pool;
   p.page_table = page_table;
   p.seq_lens = seq_lens;
   const size_t rows = static_cast<size_t>(N) * Hq * geo.max_splits;
@@ -486,12 +528,14 @@ cudaError_t launch_decode_paged(const void* q, const void* k_pool, const void* v
   p.split_tokens = geo.split_tokens;
   p.max_splits = geo.max_splits;
   p.window = window;
-  p.scale_log2 = scale * 1.4426950408889634f;
+  p.scale_log2 = scale * k_scale * 1.4426950408889634f;
+  p.v_scale = v_scale;
   p.out = static_cast<__nv_bfloat16*>(out);
   const int G = Hq / Hkv;
   cudaError_t e = cudaErrorInvalidValue;
-#define ATTN_DECODE_CASE(DD, GG) \
-  if (D == DD && G == GG) e = launch_split<DD, GG>(p, N, stream);
+#define ATTN_DECODE_CASE(DD, GG)                                        \
+  if (D == DD && G == GG)                                               \
+    e = fp8 ? launch_split<DD, GG, true>(p, N, stream) : launch_split<DD, GG, false>(p, N, stream);
   ATTN_DECODE_CASE(128, 1) ATTN_DECODE_CASE(128, 2) ATTN_DECODE_CASE(128, 4) ATTN_DECODE_CASE(128, 8)
   ATTN_DECODE_CASE(64, 1) ATTN_DECODE_CASE(64, 2) ATTN_DECODE_CASE(64, 4) ATTN_DECODE_CASE(64, 8)
 #undef ATTN_DECODE_CASE

@@ -130,3 +130,33 @@ def paged_inputs(N, Hq, Hkv, D, page_size: int, seed: int, *, seq_lens=None,
         v_pool = v_pool.masked_fill(bad[:, None, :, None].expand(total, Hkv, page_size, D), nan)
     return PagedInputs(q, k_pool.contiguous(), v_pool.contiguous(), table,
                        seq_lens.to(torch.int32), page_size, used, seed)
+
+
+def e4m3_codes(shape, seed: int, scale: float) -> torch.Tensor:
+    """N(0, 1) float32 draws from ``seed``, divided by ``scale`` and rounded to FP8 E4M3 codes (uint8).
+
+    The rounding is torch's float8_e4m3fn conversion, saturated at +-448; a
+    code stands for ``scale * value(code)``.
+    """
+    x = torch.randn(tuple(shape), generator=_gen(seed), dtype=torch.float32) / float(scale)
+    return x.clamp(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8).contiguous()
+
+
+NAN_E4M3 = 0x7F
+
+
+def paged_inputs_fp8(N, Hq, Hkv, D, page_size: int, seed: int, *, k_scale: float, v_scale: float, **kw):
+    """``paged_inputs`` with the pools replaced by E4M3 codes (``k_scale``, ``v_scale`` per pool).
+
+    The page tables, lengths and bf16 queries are those of ``paged_inputs``
+    with the same arguments; with ``poison`` every slot that must never be
+    read holds the NaN code 0x7F.
+    """
+    p = paged_inputs(N, Hq, Hkv, D, page_size, seed, **kw)
+    base = int(seed) * 16
+    k = e4m3_codes(p.k_pool.shape, base + 5, k_scale)
+    v = e4m3_codes(p.v_pool.shape, base + 6, v_scale)
+    bad = torch.isnan(p.k_pool.float())
+    k = torch.where(bad, torch.full_like(k, NAN_E4M3), k)
+    v = torch.where(bad, torch.full_like(v, NAN_E4M3), v)
+    return PagedInputs(p.q, k, v, p.page_table, p.seq_lens, page_size, p.used_pages, seed)

@@ -190,3 +190,19 @@ def test_library_needs_no_cxx_runtime_and_loads_first():
     out = subprocess.run([sys.executable, "-S", "-c", code], capture_output=True, text=True, timeout=60)
     assert out.returncode == 0, out.stderr
     assert int(out.stdout.strip()) >= 100
+
+
+def test_fp8_decode_argument_validation():
+    lib = _lib()
+
+    def call(ks=0.5, vs=0.5, D=128, Hq=8, Hkv=2, ws=FAKE, kp=FAKE):
+        return lib.attn_decode_paged_fp8(FAKE, kp, FAKE, FAKE, FAKE, 16, 4, Hq, Hkv, D, 64, 16, 256, 0.1, ks, vs, 0,
+                                         ws, 1 << 30, FAKE, None)
+    assert call(ks=0.0) == 1
+    assert call(vs=-1.0) == 1
+    assert call(ks=float("nan")) == 1
+    assert call(kp=None) == 1
+    assert call(kp=MISALIGNED) == 1
+    assert call(D=96) == 2
+    assert call(Hq=24, Hkv=2) == 2
+    assert call(ws=None) == 6

@@ -1,0 +1,91 @@
+"""GPU parity of the paged decode over an 8-bit (FP8 E4M3) cache against the float64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+from conftest import assert_parity
+from oracle import fp8, sdpa
+from scaled_dot_product_prefill_b200 import api, inputs, workloads
+
+pytestmark = pytest.mark.gpu
+
+
+def oracle_fp8(p, k_scale, v_scale, scale, window):
+    """Decode each code to the value it stands for, then the plain definition."""
+    K = fp8.dequantize(p.k_pool, k_scale)
+    V = fp8.dequantize(p.v_pool, v_scale)
+    return sdpa.decode_paged(p.q, K, V, p.page_table, p.seq_lens, p.page_size, scale, window)
+
+
+def run_fp8(p, k_scale, v_scale, window=0, scale=None):
+    dev = [t.cuda() for t in (p.q, p.k_pool, p.v_pool, p.page_table, p.seq_lens)]
+    out = api.attn_decode_paged_fp8(*dev, max_seq_len=max(p.max_seq_len, 1), k_scale=k_scale, v_scale=v_scale,
+                                    scale=scale, window=window)
+    torch.cuda.synchronize()
+    return out
+
+
+CASES = [
+    # N, Hq, Hkv, D, page, seq_lens, window, k_scale, v_scale
+    (4, 8, 2, 128, 16, [1, 16, 17, 300], 0, 1 / 64, 1 / 64),
+    (3, 4, 4, 64, 16, [5, 513, 1000], 0, 0.02, 0.03),
+    (2, 8, 1, 128, 32, [700, 33], 0, 1 / 32, 0.011),            # MQA, 32-token pages
+    (3, 16, 2, 128, 64, [2000, 64, 65], 0, 0.015, 0.015),       # group of 8
+    (3, 16, 2, 64, 16, [900, 1, 130], 0, 0.05, 0.01),           # group of 8 at D = 64
+    (4, 8, 2, 128, 16, [300, 1200, 20, 4000], 100, 1 / 64, 0.02),   # sliding window
+    (2, 8, 4, 64, 16, [1, 0], 0, 1.0, 1.0),                     # an empty cache gives zeros
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[str(c[:6]) for c in CASES])
+def test_fp8_decode_matches_oracle(case):
+    N, Hq, Hkv, D, page, lens, window, ks, vs = case
+    p = inputs.paged_inputs_fp8(N, Hq, Hkv, D, page, seed=len(lens) * 11 + D, k_scale=ks, v_scale=vs,
+                                seq_lens=lens, spare_pages=3, poison=True)
+    out = run_fp8(p, ks, vs, window)
+    assert api.attn_device_status(clear=True) == 0
+    ref = oracle_fp8(p, ks, vs, 1 / np.sqrt(D), window)
+    assert_parity(out, ref, "bf16", str(case))
+
+
+def test_fp8_decode_equals_bf16_decode_of_the_decoded_cache():
+    """With power-of-two scales every decoded element is exact in bf16 and every scaling is exact in fp32:
+    the 8-bit path must then return the bf16 path's output bit for bit."""
+    ks, vs = 1 / 64, 1 / 128
+    p = inputs.paged_inputs_fp8(6, 32, 8, 128, 16, seed=5, k_scale=ks, v_scale=vs,
+                                seq_lens=[33, 1000, 17, 4097, 250, 64])
+    K = torch.from_numpy(fp8.dequantize(p.k_pool, ks)).to(torch.bfloat16)
+    V = torch.from_numpy(fp8.dequantize(p.v_pool, vs)).to(torch.bfloat16)
+    assert torch.equal(K.double(), torch.from_numpy(fp8.dequantize(p.k_pool, ks)))   # exact in bf16
+    out8 = run_fp8(p, ks, vs)
+    dev = [t.cuda() for t in (p.q, K, V, p.page_table, p.seq_lens)]
+    out16 = api.attn_decode_paged(*dev, max_seq_len=p.max_seq_len)
+    torch.cuda.synchronize()
+    assert torch.equal(out8, out16)
+
+
+def test_fp8_decode_workload_shape_on_sampled_sequences():
+    spec = workloads.WORKLOADS["paged_decode_gqa"]
+    ks, vs = 1 / 64, 1 / 64
+    p = inputs.paged_inputs_fp8(spec.N, spec.Hq, spec.Hkv, spec.D, spec.page_size, spec.seed, k_scale=ks,
+                                v_scale=vs, len_range=spec.len_range)
+    out = run_fp8(p, ks, vs, spec.window, spec.scale).cpu()
+    assert api.attn_device_status(clear=True) == 0
+    for b in (0, 1, spec.N // 2, spec.N - 1):
+        L = int(p.seq_lens[b])
+        K = fp8.dequantize(sdpa.gather_pages(p.k_pool.numpy(), p.page_table[b].numpy(), L, spec.page_size), ks)
+        V = fp8.dequantize(sdpa.gather_pages(p.v_pool.numpy(), p.page_table[b].numpy(), L, spec.page_size), vs)
+        ref = sdpa.attention(p.q[b][None, :, None, :], K.transpose(1, 0, 2)[None], V.transpose(1, 0, 2)[None],
+                             spec.scale, causal=True)[0, :, 0]
+        assert_parity(out[b], ref, "bf16", f"{spec.name} fp8 seq {b}")
+
+
+def test_fp8_decode_rejects_bad_scales_and_dtypes():
+    p = inputs.paged_inputs_fp8(2, 8, 2, 128, 16, seed=1, k_scale=1.0, v_scale=1.0, seq_lens=[20, 40])
+    with pytest.raises(api.AttnError):
+        run_fp8(p, 0.0, 1.0)
+    with pytest.raises(api.AttnError):
+        run_fp8(p, 1.0, float("inf"))
+    with pytest.raises(ValueError):
+        api.attn_decode_paged_fp8(p.q.cuda(), p.k_pool.cuda().view(torch.int8), p.v_pool.cuda(),
+                                  p.page_table.cuda(), p.seq_lens.cuda(), max_seq_len=40, k_scale=1, v_scale=1)

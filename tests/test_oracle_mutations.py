@@ -9,7 +9,7 @@ import numpy as np
 import pytest
 
 import test_oracle_pins as pins
-from oracle import sdpa
+from oracle import fp8, sdpa
 
 _orig_visible = sdpa.visible
 _orig_softmax = sdpa.softmax_rows
@@ -64,6 +64,19 @@ def _append_chunk_reversed(pool, page_table, seq_lens, new, page_size):
     return _orig_append(pool, page_table, seq_lens, np.asarray(new)[:, :, ::-1], page_size)
 
 
+def _e4m3_bias_8(codes):
+    return fp8.__dict__["_orig_e4m3"](codes) / 2.0
+
+
+def _e4m3_subnormals_as_normals(codes):
+    c = np.asarray(codes.numpy() if hasattr(codes, "numpy") else codes, dtype=np.uint8)
+    v = fp8.__dict__["_orig_e4m3"](c)
+    sub = ((c >> 3) & 0xF) == 0
+    return np.where(sub, np.where(c & 0x80, -1.0, 1.0) * (1 + (c & 7) / 8.0) * 2.0 ** -7, v)
+
+
+fp8.__dict__.setdefault("_orig_e4m3", fp8.e4m3_value)
+
 MUTATIONS = {
     "kv_head round robin": ("kv_head", lambda h, Hq, Hkv: h % Hkv),
     "window off by one": ("visible", _visible_window_off_by_one),
@@ -75,6 +88,8 @@ MUTATIONS = {
     "value rows reversed": ("weights", _weights_keys_reversed),
     "append one slot late": ("append_pages", _append_one_slot_late),
     "append chunk reversed": ("append_pages", _append_chunk_reversed),
+    "e4m3 exponent bias 8": ("fp8.e4m3_value", _e4m3_bias_8),
+    "e4m3 subnormals read as normals": ("fp8.e4m3_value", _e4m3_subnormals_as_normals),
 }
 
 PIN_TESTS = [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]
@@ -96,7 +111,10 @@ def _run_pin(fn):
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
 def test_pins_catch_planted_mistake(name, monkeypatch):
     attr, bad = MUTATIONS[name]
-    monkeypatch.setattr(sdpa, attr, bad)
+    if attr.startswith("fp8."):
+        monkeypatch.setattr(fp8, attr[4:], bad)
+    else:
+        monkeypatch.setattr(sdpa, attr, bad)
     caught = []
     for fn in PIN_TESTS:
         if fn.__name__ in ("test_scale_table_statistics",):

@@ -390,3 +390,37 @@ def test_append_then_decode_equals_full_causal_recompute():
         v_pool = sdpa.append_pages(v_pool, table, [t + 1], v[:, :, t:t + 1], page)
         step = sdpa.decode_paged(q[0, :, t][None], k_pool, v_pool, table, [t + 1], page, 0.3)
         np.testing.assert_allclose(step[0], full[0, :, t], atol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# 8-bit codes of the fp8 cache
+
+
+def test_e4m3_values_at_the_format_landmarks():
+    from oracle import fp8
+
+    v = fp8.e4m3_value(np.array([0x00, 0x80, 0x01, 0x07, 0x08, 0x38, 0xB8, 0x3C, 0x7E, 0xFE, 0x7F, 0xFF], np.uint8))
+    want = [0.0, -0.0, 2.0 ** -9, 7 * 2.0 ** -9, 2.0 ** -6, 1.0, -1.0, 1.5, 448.0, -448.0]
+    np.testing.assert_array_equal(v[:10], want)
+    assert np.signbit(v[1])
+    assert np.isnan(v[10]) and np.isnan(v[11])
+    # the positive finite codes are strictly increasing; the step up from code c is one ulp of
+    # c's binade, 2^(max(e, 1) - 10) for exponent field e (subnormals share the first binade's ulp)
+    pos = fp8.e4m3_value(np.arange(0x7F, dtype=np.uint8))
+    steps = np.diff(pos)
+    assert (steps > 0).all()
+    e = np.maximum(np.arange(0, 0x7E) >> 3, 1)
+    np.testing.assert_array_equal(steps, 2.0 ** (e - 10.0))
+
+
+def test_e4m3_values_match_torch_float8_for_every_code():
+    import torch
+
+    from oracle import fp8
+
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = fp8.e4m3_value(codes)
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    np.testing.assert_array_equal(got[ok], ref[ok])
