@@ -387,6 +387,21 @@ attn_status_t attn_kv_append(const void* k_new, const void* v_new, void* k_pool,
                              int page_size, int B, int Hkv, int S_new, int D,
                              int num_pages, int max_pages, attn_stream_t stream);
 
+/*
+ * attn_kv_append_fp8 -- attn_kv_append into an 8-bit cache (the pools of
+ * attn_decode_paged_fp8).  Each bf16 element x of k_new (v_new) becomes the
+ * E4M3 code nearest to x * (1 / k_scale) (v_scale): the reciprocal and the
+ * product are rounded to float32, the code to nearest with ties to the even
+ * code, and magnitudes above 448 saturate to +-448 (cvt.rn.satfinite).
+ * k_pool, v_pool: [num_pages, Hkv, page_size, D] uint8.  k_scale, v_scale:
+ * finite and > 0.  Everything else, the errors included, is as attn_kv_append.
+ */
+attn_status_t attn_kv_append_fp8(const void* k_new, const void* v_new, uint8_t* k_pool, uint8_t* v_pool,
+                                 const int32_t* page_table, const int32_t* seq_lens,
+                                 int page_size, int B, int Hkv, int S_new, int D,
+                                 int num_pages, int max_pages, float k_scale, float v_scale,
+                                 attn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -15,7 +15,8 @@ from ._lib import AttnError
 
 __all__ = ["attn_prefill", "attn_prefill_f32", "attn_prefill_lse", "attn_prefill_f32_lse",
            "attn_prefill_paged", "attn_decode_paged", "attn_decode_paged_noalloc",
-           "attn_decode_paged_workspace_size", "attn_decode_paged_fp8", "attn_kv_append", "PagePool",
+           "attn_decode_paged_workspace_size", "attn_decode_paged_fp8", "attn_kv_append", "attn_kv_append_fp8",
+           "PagePool",
            "attn_device_status", "attn_status_string", "attn_version", "AttnError"]
 
 
@@ -234,6 +235,26 @@ def attn_kv_append(k_new, v_new, k_pool, v_pool, page_table, seq_lens, *, stream
     _check("attn_kv_append", _lib.load().attn_kv_append(
         _ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool), _ptr(page_table), _ptr(seq_lens), page_size, B, Hkv,
         S_new, D, num_pages, page_table.shape[1], _stream(stream)))
+
+
+def attn_kv_append_fp8(k_new, v_new, k_pool, v_pool, page_table, seq_lens, *, k_scale, v_scale, stream=None):
+    """attn_kv_append into uint8 E4M3 pools: code = nearest E4M3 to x * (1/scale) (float32, ties to even)."""
+    B, Hkv, S_new, D = k_new.shape
+    num_pages, Hkv_p, page_size, D_p = k_pool.shape
+    if tuple(v_new.shape) != tuple(k_new.shape) or tuple(v_pool.shape) != tuple(k_pool.shape):
+        raise ValueError("k_new/v_new and k_pool/v_pool must have matching shapes")
+    if Hkv_p != Hkv or D_p != D:
+        raise ValueError("the pools' head count and head dim must match k_new")
+    if k_new.dtype != torch.bfloat16 or v_new.dtype != torch.bfloat16:
+        raise ValueError("k_new and v_new must be bfloat16")
+    if k_pool.dtype != torch.uint8 or v_pool.dtype != torch.uint8:
+        raise ValueError("the pools must hold uint8 E4M3 codes")
+    _need_cuda(k_new, v_new, k_pool, v_pool, page_table, seq_lens)
+    if page_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise ValueError("page_table and seq_lens must be int32")
+    _check("attn_kv_append_fp8", _lib.load().attn_kv_append_fp8(
+        _ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool), _ptr(page_table), _ptr(seq_lens), page_size, B, Hkv,
+        S_new, D, num_pages, page_table.shape[1], float(k_scale), float(v_scale), _stream(stream)))
 
 
 class PagePool:

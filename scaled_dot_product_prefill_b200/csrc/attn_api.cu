@@ -269,10 +269,16 @@ attn_status_t attn_decode_paged_noalloc(const void* q, const void* k_pool, const
                            max_seq_len, scale, window, scratch, attn::decode_scratch_capacity(), out, stream);
 }
 
-attn_status_t attn_kv_append(const void* k_new, const void* v_new, void* k_pool, void* v_pool,
-                             const int32_t* page_table, const int32_t* seq_lens, int page_size, int B, int Hkv,
-                             int S_new, int D, int num_pages, int max_pages, attn_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+attn_status_t kv_append(const void* k_new, const void* v_new, void* k_pool, void* v_pool, const int32_t* page_table,
+                        const int32_t* seq_lens, int page_size, int B, int Hkv, int S_new, int D, int num_pages,
+                        int max_pages, attn_stream_t stream, bool fp8, float k_scale, float v_scale) {
   if (B < 0 || Hkv < 0 || S_new < 0 || D <= 0 || page_size <= 0 || num_pages < 0 || max_pages < 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (!(k_scale > 0.f) || !std::isfinite(k_scale) || !(v_scale > 0.f) || !std::isfinite(v_scale))
     return ATTN_ERR_INVALID_ARG;
   if (B == 0 || Hkv == 0 || S_new == 0) return ATTN_OK;
   if (k_new == nullptr || v_new == nullptr || k_pool == nullptr || v_pool == nullptr || page_table == nullptr ||
@@ -285,7 +291,26 @@ attn_status_t attn_kv_append(const void* k_new, const void* v_new, void* k_pool,
   if (static_cast<long long>(B) * Hkv * S_new * (D / 8) > 0x7FFFFFFFLL) return ATTN_ERR_UNSUPPORTED;
   return from_cuda(attn::launch_kv_append(k_new, v_new, k_pool, v_pool, page_table, seq_lens, page_size, B, Hkv,
                                           S_new, D, num_pages, max_pages, attn::device_error_word(),
-                                          reinterpret_cast<cudaStream_t>(stream)));
+                                          reinterpret_cast<cudaStream_t>(stream), fp8, k_scale, v_scale));
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status_t attn_kv_append(const void* k_new, const void* v_new, void* k_pool, void* v_pool,
+                             const int32_t* page_table, const int32_t* seq_lens, int page_size, int B, int Hkv,
+                             int S_new, int D, int num_pages, int max_pages, attn_stream_t stream) {
+  return kv_append(k_new, v_new, k_pool, v_pool, page_table, seq_lens, page_size, B, Hkv, S_new, D, num_pages,
+                   max_pages, stream, false, 1.f, 1.f);
+}
+
+attn_status_t attn_kv_append_fp8(const void* k_new, const void* v_new, uint8_t* k_pool, uint8_t* v_pool,
+                                 const int32_t* page_table, const int32_t* seq_lens, int page_size, int B, int Hkv,
+                                 int S_new, int D, int num_pages, int max_pages, float k_scale, float v_scale,
+                                 attn_stream_t stream) {
+  return kv_append(k_new, v_new, k_pool, v_pool, page_table, seq_lens, page_size, B, Hkv, S_new, D, num_pages,
+                   max_pages, stream, true, k_scale, v_scale);
 }
 
 attn_status_t attn_device_status(int clear) {

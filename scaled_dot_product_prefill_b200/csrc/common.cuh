@@ -57,6 +57,7 @@ cudaError_t launch_decode_paged(const void* q, const void* k_pool, const void* v
 // k_new/v_new [B, Hkv, S_new, D] -> pools [num_pages, Hkv, page_size, D] at positions seq_lens[b] - S_new + i.
 cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* k_pool, void* v_pool,
                              const int32_t* page_table, const int32_t* seq_lens, int page_size, int B, int Hkv,
-                             int S_new, int D, int num_pages, int max_pages, unsigned int* err, cudaStream_t stream);
+                             int S_new, int D, int num_pages, int max_pages, unsigned int* err, cudaStream_t stream,
+                             bool fp8 = false, float k_scale = 1.f, float v_scale = 1.f);
 
 }  // namespace attn

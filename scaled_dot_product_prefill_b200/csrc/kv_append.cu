@@ -37,13 +37,33 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
 constexpr int kThreads = 256;
 constexpr int kUnroll = ATTN_APPEND_UNROLL;   // pieces per thread per pass, all loads issued before any store
 
+// 8 bf16 -> 8 FP8 E4M3 codes of x * inv_scale, rounded to nearest even and
+// saturated at +-448 (cvt.rn.satfinite); element 0 lands in the lowest byte.
+__device__ __forceinline__ uint2 quantize8_e4m3(const uint4& u, float inv_scale) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  uint32_t out[2] = {0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float x0 = __uint_as_float(w[i] << 16) * inv_scale;
+    const float x1 = __uint_as_float(w[i] & 0xFFFF0000u) * inv_scale;
+    unsigned short pair;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pair) : "f"(x1), "f"(x0));   // x1 high, x0 low
+    out[i >> 1] |= static_cast<uint32_t>(pair) << (16 * (i & 1));
+  }
+  return make_uint2(out[0], out[1]);
+}
+
+// FP8: the pools hold E4M3 codes and each 16-byte piece of a bf16 row becomes
+// 8 bytes of codes (k * k_inv, v * v_inv).
+template <bool FP8>
 __global__ void __launch_bounds__(kThreads) kv_append_kernel(const uint4* __restrict__ k_new,
                                                              const uint4* __restrict__ v_new,
-                                                             uint4* __restrict__ k_pool, uint4* __restrict__ v_pool,
+                                                             void* __restrict__ k_pool, void* __restrict__ v_pool,
                                                              const int32_t* __restrict__ page_table,
                                                              const int32_t* __restrict__ seq_lens, int page_size,
                                                              int B, int Hkv, int S_new, int pieces, int num_pages,
-                                                             int max_pages, unsigned int* err) {
+                                                             int max_pages, unsigned int* err, float k_inv,
+                                                             float v_inv) {
   const unsigned int total = static_cast<unsigned int>(B) * Hkv * S_new * pieces;
   const unsigned int pass = gridDim.x * kThreads * kUnroll;
   for (unsigned int base = blockIdx.x * kThreads * kUnroll + threadIdx.x; base < total; base += pass) {
@@ -81,8 +101,13 @@ __global__ void __launch_bounds__(kThreads) kv_append_kernel(const uint4* __rest
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       if (!ok[u]) continue;
-      k_pool[dst[u]] = kv[u];
-      v_pool[dst[u]] = vv[u];
+      if constexpr (FP8) {
+        static_cast<uint2*>(k_pool)[dst[u]] = quantize8_e4m3(kv[u], k_inv);
+        static_cast<uint2*>(v_pool)[dst[u]] = quantize8_e4m3(vv[u], v_inv);
+      } else {
+        static_cast<uint4*>(k_pool)[dst[u]] = kv[u];
+        static_cast<uint4*>(v_pool)[dst[u]] = vv[u];
+      }
     }
   }
 }
@@ -91,7 +116,8 @@ __global__ void __launch_bounds__(kThreads) kv_append_kernel(const uint4* __rest
 
 cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* k_pool, void* v_pool,
                              const int32_t* page_table, const int32_t* seq_lens, int page_size, int B, int Hkv,
-                             int S_new, int D, int num_pages, int max_pages, unsigned int* err, cudaStream_t stream) {
+                             int S_new, int D, int num_pages, int max_pages, unsigned int* err, cudaStream_t stream,
+                             bool fp8, float k_scale, float v_scale) {
   static int sms[64] = {0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -106,9 +132,10 @@ cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* k_pool,
   // one pass of resident blocks (8 x 256 threads per SM) covers up to 8 * n_sm * 256 * kUnroll pieces
   const long long want = (total + kThreads * kUnroll - 1) / (kThreads * kUnroll);
   const int grid = static_cast<int>(want < 8LL * n_sm ? want : 8LL * n_sm);
-  kv_append_kernel<<<grid, kThreads, 0, stream>>>(
-      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), static_cast<uint4*>(k_pool),
-      static_cast<uint4*>(v_pool), page_table, seq_lens, page_size, B, Hkv, S_new, pieces, num_pages, max_pages, err);
+  auto kern = fp8 ? kv_append_kernel<true> : kv_append_kernel<false>;
+  kern<<<grid, kThreads, 0, stream>>>(static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), k_pool,
+                                      v_pool, page_table, seq_lens, page_size, B, Hkv, S_new, pieces, num_pages,
+                                      max_pages, err, 1.f / k_scale, 1.f / v_scale);
   return cudaGetLastError();
 }
 

@@ -206,3 +206,14 @@ def test_fp8_decode_argument_validation():
     assert call(D=96) == 2
     assert call(Hq=24, Hkv=2) == 2
     assert call(ws=None) == 6
+
+
+def test_fp8_append_argument_validation():
+    lib = _lib()
+
+    def call(ks=0.5, vs=0.5, D=128, kp=FAKE):
+        return lib.attn_kv_append_fp8(FAKE, FAKE, kp, FAKE, FAKE, FAKE, 16, 2, 2, 4, D, 8, 4, ks, vs, None)
+    assert call(ks=0.0) == 1
+    assert call(vs=float("inf")) == 1
+    assert call(kp=None) == 1
+    assert call(D=100) == 2

@@ -89,3 +89,49 @@ def test_fp8_decode_rejects_bad_scales_and_dtypes():
     with pytest.raises(ValueError):
         api.attn_decode_paged_fp8(p.q.cuda(), p.k_pool.cuda().view(torch.int8), p.v_pool.cuda(),
                                   p.page_table.cuda(), p.seq_lens.cuda(), max_seq_len=40, k_scale=1, v_scale=1)
+
+
+def bits8(t):
+    return t.cpu().numpy()
+
+
+@pytest.mark.parametrize("ks,vs", [(0.05, 0.013), (1 / 64, 1 / 32)])
+def test_fp8_append_matches_the_oracle_quantizer_bit_for_bit(ks, vs):
+    B, Hkv, S_new, D, page = 3, 2, 40, 128, 16
+    lens = [40, 100, 23]                       # sequence 2 is shorter than the chunk
+    p = inputs.paged_inputs_fp8(B, 1, Hkv, D, page, seed=17, k_scale=1.0, v_scale=1.0, seq_lens=lens,
+                                spare_pages=2, poison=True)
+    k_new = (inputs.normal((B, Hkv, S_new, D), seed=3).float() * 4).to(torch.bfloat16)   # some saturate
+    v_new = inputs.normal((B, Hkv, S_new, D), seed=4)
+    kp, vp = p.k_pool.cuda(), p.v_pool.cuda()
+    api.attn_device_status(clear=True)
+    api.attn_kv_append_fp8(k_new.cuda(), v_new.cuda(), kp, vp, p.page_table.cuda(), p.seq_lens.cuda(),
+                           k_scale=ks, v_scale=vs)
+    torch.cuda.synchronize()
+    assert api.attn_device_status(clear=True) == 0
+    table, sl = p.page_table.numpy(), p.seq_lens.numpy()
+    want_k = sdpa.append_pages(p.k_pool.numpy(), table, sl, fp8.quantize(k_new, ks), page)
+    want_v = sdpa.append_pages(p.v_pool.numpy(), table, sl, fp8.quantize(v_new, vs), page)
+    np.testing.assert_array_equal(bits8(kp), want_k)
+    np.testing.assert_array_equal(bits8(vp), want_v)
+
+
+def test_fp8_cache_filled_by_the_append_decodes_like_the_oracle():
+    """Prefill-time append of whole caches into 8-bit pools, then a decode step against them."""
+    N, Hq, Hkv, D, page, L = 4, 16, 4, 128, 16, 777
+    ks, vs = 0.02, 0.02
+    p = inputs.paged_inputs_fp8(N, Hq, Hkv, D, page, seed=23, k_scale=ks, v_scale=vs, seq_lens=[L] * N,
+                                poison=True)
+    k_new = inputs.normal((N, Hkv, L, D), seed=8)
+    v_new = inputs.normal((N, Hkv, L, D), seed=9)
+    kp = torch.full_like(p.k_pool, inputs.NAN_E4M3).cuda()
+    vp = torch.full_like(p.v_pool, inputs.NAN_E4M3).cuda()
+    pt, sl = p.page_table.cuda(), p.seq_lens.cuda()
+    api.attn_kv_append_fp8(k_new.cuda(), v_new.cuda(), kp, vp, pt, sl, k_scale=ks, v_scale=vs)
+    out = api.attn_decode_paged_fp8(p.q.cuda(), kp, vp, pt, sl, max_seq_len=L, k_scale=ks, v_scale=vs)
+    torch.cuda.synchronize()
+    assert api.attn_device_status(clear=True) == 0
+    K = fp8.dequantize(fp8.quantize(k_new, ks), ks)          # [N, Hkv, L, D]
+    V = fp8.dequantize(fp8.quantize(v_new, vs), vs)
+    ref = sdpa.attention(p.q.double().numpy()[:, :, None, :], K, V, 1 / np.sqrt(D), causal=True)[:, :, 0]
+    assert_parity(out, ref, "bf16", "fp8 cache from the append")

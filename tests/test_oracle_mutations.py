@@ -75,7 +75,18 @@ def _e4m3_subnormals_as_normals(codes):
     return np.where(sub, np.where(c & 0x80, -1.0, 1.0) * (1 + (c & 7) / 8.0) * 2.0 ** -7, v)
 
 
+def _e4m3_ties_away(x):
+    x = np.asarray(x, dtype=np.float64)
+    got = fp8.__dict__["_orig_round"](x)
+    up = fp8.__dict__["_orig_round"](np.nextafter(np.abs(x), np.inf)) & 0x7F
+    v = fp8.e4m3_value(got & 0x7F)
+    nxt = fp8.e4m3_value(np.minimum((got & 0x7F) + 1, 0x7E))
+    tie = np.abs(np.abs(x) - (v + nxt) / 2) == 0
+    return np.where(tie, up | (got & 0x80), got).astype(np.uint8)
+
+
 fp8.__dict__.setdefault("_orig_e4m3", fp8.e4m3_value)
+fp8.__dict__.setdefault("_orig_round", fp8.e4m3_round)
 
 MUTATIONS = {
     "kv_head round robin": ("kv_head", lambda h, Hq, Hkv: h % Hkv),
@@ -90,6 +101,7 @@ MUTATIONS = {
     "append chunk reversed": ("append_pages", _append_chunk_reversed),
     "e4m3 exponent bias 8": ("fp8.e4m3_value", _e4m3_bias_8),
     "e4m3 subnormals read as normals": ("fp8.e4m3_value", _e4m3_subnormals_as_normals),
+    "e4m3 ties rounded away from zero": ("fp8.e4m3_round", _e4m3_ties_away),
 }
 
 PIN_TESTS = [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]

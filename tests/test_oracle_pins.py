@@ -424,3 +424,32 @@ def test_e4m3_values_match_torch_float8_for_every_code():
     np.testing.assert_array_equal(np.isnan(got), np.isnan(ref))
     ok = ~np.isnan(ref)
     np.testing.assert_array_equal(got[ok], ref[ok])
+
+
+def test_e4m3_rounding_round_trips_ties_to_even_and_saturates():
+    from oracle import fp8
+
+    codes = np.arange(256, dtype=np.uint8)
+    codes = codes[(codes & 0x7F) != 0x7F]
+    np.testing.assert_array_equal(fp8.e4m3_round(fp8.e4m3_value(codes)), codes)
+    pos = fp8.e4m3_value(np.arange(0x7F, dtype=np.uint8))
+    mid = (pos[:-1] + pos[1:]) / 2                       # exact halfway points (in float64)
+    got = fp8.e4m3_round(mid)
+    lower = np.arange(0x7E)
+    np.testing.assert_array_equal(got, np.where(lower % 2 == 0, lower, lower + 1))
+    eps = np.diff(pos) / 8
+    np.testing.assert_array_equal(fp8.e4m3_round(mid - eps), lower)
+    np.testing.assert_array_equal(fp8.e4m3_round(mid + eps), lower + 1)
+    np.testing.assert_array_equal(fp8.e4m3_round([448.0, 449.0, 1e30, -1e30, -0.0, -1e-9]),
+                                  [0x7E, 0x7E, 0x7E, 0xFE, 0x80, 0x80])
+
+
+def test_e4m3_rounding_matches_torch_float8_in_range():
+    import torch
+
+    from oracle import fp8
+
+    x = np.float32(np.random.default_rng(3).standard_normal(200000) * 60)
+    x = x[np.abs(x) <= 448]
+    want = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(fp8.e4m3_round(x), want)
