@@ -56,6 +56,9 @@ constexpr int kMmaWarp = 9;
 // and MMA warps, two idle warps) gets kProducerRegs.  The split must fit the
 // launch allocation: 128 * (2 * kSoftmaxRegs + kProducerRegs) <= kThreads *
 // regs-per-thread at launch, which the host checks before every launch.
+#ifndef ATTN_PREFILL_TURNS
+#define ATTN_PREFILL_TURNS 0
+#endif
 constexpr int kSoftmaxRegs = 208;
 constexpr int kProducerRegs = 88;
 constexpr uint32_t kTmemCols = 512;
@@ -80,6 +83,11 @@ struct Cfg {
   // computed while the softmax of tile j is still running.  D = 128 has no
   // room: P_i is written over the first 64 columns of S_i, O_i [256 + 128 i, +128).
   static constexpr bool SEP_P = (D == 64);
+  // TURNS: the two softmax groups take turns at the exponentials, so that one
+  // group's exponentials run at the full MUFU rate while the other loads S,
+  // takes its row max and stores P (ATTN_PREFILL_TURNS: 0 never, 1 at D = 64,
+  // 2 always).
+  static constexpr bool TURNS = (ATTN_PREFILL_TURNS == 2) || (ATTN_PREFILL_TURNS == 1 && D == 64);
   static constexpr uint32_t S_COL = 0;                // + 128 * i
   static constexpr uint32_t P_COL = SEP_P ? 256 : 0;  // + (SEP_P ? 64 : 128) * i
   static constexpr uint32_t P_STRIDE = SEP_P ? 64 : 128;
@@ -200,7 +208,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* o_done = p_ready + NQ;                      // NQ: O_i final (SEP_P: each P_i V done)
   uint64_t* s_free = o_done + NQ;                       // NQ: S_i loaded by the softmax (SEP_P)
   uint64_t* drain = s_free + NQ;                        // 1
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* turn = drain + 1;                           // NQ: group i may run its exponentials (TURNS)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(turn + NQ);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -220,6 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&p_ready[i], 4 * 32);
       mbar_init(&o_done[i], 1);
       mbar_init(&s_free[i], 4 * 32);
+      mbar_init(&turn[i], 4 * 32);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -515,6 +525,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
     int t = 0, oc = 0;
     int pv = 0;   // SEP_P: P_i V products of this tile completed and waited for
+    // Turns at the exponentials (TURNS): group 0 goes first; each group waits
+    // for its turn, runs its exponentials and hands the turn over.  Both groups
+    // take the same number of turns per item: the one with fewer key tiles
+    // takes empty turns first.  Group 1 opens group 0's first turn.
+    int tk = 0;   // turns this group has waited for
+    if constexpr (C::TURNS) {
+      if (i == 1) mbar_arrive(&turn[0]);
+    }
+    auto take_turn = [&]() -> bool {
+      const bool r = mbar_wait(&turn[i], tk & 1, abort_flag, p.err);
+      ++tk;
+      return __all_sync(0xffffffffu, r);
+    };
+    auto pass_turn = [&]() { mbar_arrive(&turn[1 - i]); };
     // O_i *= alpha (every row of the warp takes part when any row needs it)
     auto rescale_o = [&](bool later_tile, float alpha) {
       if (!__any_sync(0xffffffffu, later_tile && alpha != 1.f)) return;
@@ -542,6 +566,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Item it = make_item<PAGED>(p, k);
       const int my_lo = (i == 0) ? it.lo[0] : it.lo[1];
       const int my_hi = (i == 0) ? it.hi[0] : it.hi[1];
+      if constexpr (C::TURNS) {
+        const int n_mine = max(0, my_hi - my_lo);
+        const int n_other = (i == 0) ? max(0, it.hi[1] - it.lo[1]) : max(0, it.hi[0] - it.lo[0]);
+        for (int e = n_mine; e < n_other && ok; ++e) {
+          ok = take_turn();
+          if (ok) pass_turn();
+        }
+        if (!ok) break;
+      }
       const int r0 = it.q_row0 + BM * i;
       const int r = r0 + rl;                 // query row of this thread
       const bool store = r < p.Sq;
@@ -596,6 +629,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_ref = m_tile;
         }
         if constexpr (!C::SEP_P) rescale_o(j > my_lo, alpha);   // O_i is current: S_i(j) covers P_i V(j-1)
+        if constexpr (C::TURNS) {
+          if (!(ok = take_turn())) break;
+        }
         const float mb = (m_ref == -INFINITY) ? 0.f : m_ref;
         const uint64_t nm2 = f2_pack(-mb, -mb);
         uint32_t pk[BN / 2];
@@ -621,6 +657,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         f2_unpack(f2_add(sum2[0], sum2[1]), s0, s1);
         f2_unpack(f2_add(sum2[2], sum2[3]), s2, s3);
         l += (s0 + s1) + (s2 + s3);
+        if constexpr (C::TURNS) pass_turn();
         // The exponentials above need nothing from tensor memory; only now must
         // P_i(j-1) V be complete: before O_i is rescaled and (separate P) before
         // P_i is rewritten.  Waiting here hides that product behind them.
