@@ -169,6 +169,26 @@ def oracle_decode_sample(budget_s=6.0):
 # ---------------------------------------------------------------- GPU leg
 
 
+def max_over_ranks(values, dist, device):
+    """Element-wise maximum of ``values`` over all ranks (each rank's own list when ``dist`` is None).
+
+    Every rank must call it at the same point with the same number of values.
+    """
+    values = [float(v) for v in values]
+    if dist is None:
+        return values
+    import torch
+
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_rate(units_per_rank, world, ms):
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time (weak scaling)."""
+    return world * float(units_per_rank) / (ms * 1e-3)
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
 
@@ -235,10 +255,7 @@ def run_ours(args, rank, world, local_rank):
     stats = {name: {"median": round(float(np.median(t)), 5), "mean": round(float(np.mean(t)), 5),
                     "std": round(float(np.std(t)), 5)} for name, t in (("prefill_ms", t_pre), ("decode_ms", t_dec))}
     step_ms = pre_ms + dec_ms
-    if dist is not None:
-        tt = torch.tensor([pre_ms, dec_ms, step_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        pre_ms, dec_ms, step_ms = (float(x) for x in tt.tolist())
+    pre_ms, dec_ms, step_ms = max_over_ranks([pre_ms, dec_ms, step_ms], dist, dev)
 
     # ---- end to end through the public API: pinned host inputs -> device -> kernel -> host result
     hq, hk, hv = (t.pin_memory() for t in (pi.q, pi.k, pi.v))
@@ -259,10 +276,7 @@ def run_ours(args, rank, world, local_rank):
             ev[1].record()
     torch.cuda.synchronize()
     e2e_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in e_ev]))
-    if dist is not None:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    (e2e_ms,) = max_over_ranks([e2e_ms], dist, dev)
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
     d2h = hout.numel() * hout.element_size()
 
@@ -281,7 +295,7 @@ def run_ours(args, rank, world, local_rank):
 
     result = None
     if rank == 0:
-        tflops = world * p_flops / (pre_ms * 1e-3) / 1e12
+        tflops = job_rate(p_flops, world, pre_ms) / 1e12
         peak_t = float(peaks["bf16_tflops"])
         peak_h = float(peaks["hbm_gbs"])
         ach_t = p_flops / (pre_ms * 1e-3) / 1e12
@@ -318,11 +332,11 @@ def run_ours(args, rank, world, local_rank):
                                 "frac": round(ach_d / peak_h, 4), "traffic": traffic_d,
                                 "kernel": "decode_split_kernel<128,4> + decode_combine_kernel<128>",
                                 "peak_kind": f"HBM copy, {peak_kind}"},
-            "decode": {"value": round(world * d_bytes / (dec_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+            "decode": {"value": round(job_rate(d_bytes, world, dec_ms) / 1e9, 1), "unit": "GB/s",
                        "ms": round(dec_ms, 5)},
             "prefill_ms": round(pre_ms, 5),
             "timing": dict(stats, prefill_graph_ms=None if graph_ms is None else round(graph_ms, 5)),
-            "e2e": {"value": round(world * p_flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            "e2e": {"value": round(job_rate(p_flops, world, e2e_ms) / 1e12, 3), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms": round(e2e_ms, 5),
                     "path": "pinned host q/k/v -> device, attn_prefill, out -> pinned host"},
             "gpu_launches": 3 * args.steps,
