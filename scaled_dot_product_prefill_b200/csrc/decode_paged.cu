@@ -28,7 +28,9 @@
 //   split writes its normalised partial output and base-2 log-sum-exp.
 // * decode_combine_kernel: one warp per (sequence, head) merges the splits,
 //   weighting each by 2^(lse_s - max lse) ("Attention From Scratch"
-//   README, section "Flash Attention": the pair (output, lse)).
+//   README, section "Flash Attention": the pair (output, lse)).  The lanes
+//   load 32 splits' log-sum-exps at once, and several splits' partial
+//   outputs are in flight per warp.
 #include <cmath>
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -429,7 +431,7 @@ __global__ void __launch_bounds__(kWarps * 32, (G >= 8) ? 2 : ATTN_DECODE_MINB)
 
 template <int D>
 __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams p, int N) {
-  constexpr int PER = D / 32;
+  constexpr int PER = D / 32;   // output columns per lane: 4 (one 16-byte load) or 2 (8 bytes)
   const int warp_global = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (warp_global >= N * p.Hq) return;
@@ -445,17 +447,38 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
     const int lo = (p.window > 0) ? max(0, L - p.window) : 0;
     const int s0 = lo / p.split_tokens, s1 = (L - 1) / p.split_tokens;
     const size_t rowbase = static_cast<size_t>(warp_global) * p.max_splits;
+    // the splits' log-sum-exps, 32 at a time across the lanes, and their maximum
     float M = -INFINITY;
-    for (int s = s0; s <= s1; ++s) M = fmaxf(M, p.ws_lse[rowbase + s]);
-    if (M != -INFINITY) {
-      for (int s = s0; s <= s1; ++s) {
-        const float lse = p.ws_lse[rowbase + s];
-        const float w = (lse == -INFINITY) ? 0.f : ex2(lse - M);
-        wsum += w;
-        const float* o = p.ws_o + (rowbase + s) * D;
+    for (int s = s0 + lane; s <= s1; s += 32) M = fmaxf(M, p.ws_lse[rowbase + s]);
 #pragma unroll
-        for (int t = 0; t < PER; ++t) acc[t] = fmaf(w, o[lane * PER + t], acc[t]);
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    if (M != -INFINITY) {
+      for (int base = s0; base <= s1; base += 32) {
+        const int s = base + lane;
+        const float lse = (s <= s1) ? p.ws_lse[rowbase + s] : -INFINITY;
+        const float w = (lse == -INFINITY) ? 0.f : ex2(lse - M);   // lane k holds split base + k's weight
+        wsum += w;
+        const int cnt = min(32, s1 - base + 1);
+        // independent loads of several splits' partial outputs in flight
+#pragma unroll 4
+        for (int k = 0; k < cnt; ++k) {
+          const float wk = __shfl_sync(0xffffffffu, w, k);
+          const float* o = p.ws_o + (rowbase + base + k) * D + lane * PER;
+          if constexpr (PER == 4) {
+            const float4 v = *reinterpret_cast<const float4*>(o);
+            acc[0] = fmaf(wk, v.x, acc[0]);
+            acc[1] = fmaf(wk, v.y, acc[1]);
+            acc[2] = fmaf(wk, v.z, acc[2]);
+            acc[3] = fmaf(wk, v.w, acc[3]);
+          } else {
+            const float2 v = *reinterpret_cast<const float2*>(o);
+            acc[0] = fmaf(wk, v.x, acc[0]);
+            acc[1] = fmaf(wk, v.y, acc[1]);
+          }
+        }
       }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
     }
   }
   const float inv = (wsum > 0.f) ? p.v_scale / wsum : 0.f;
