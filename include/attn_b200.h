@@ -27,6 +27,22 @@
  *                                     and "Paged KV Cache"; "LLM core
  *                                     technology", section "PagedAttention").
  *
+ * Around them:
+ *
+ *   attn_prefill_lse, attn_prefill_f32_lse   the same prefill, with each row's
+ *                                     log-sum-exp (the README's FlashAttention
+ *                                     returns the pair (output, lse)).
+ *   attn_prefill_paged                chunked prefill whose keys and values sit
+ *                                     in the paged cache.
+ *   attn_decode_paged_fp8             the decode over a cache of 8-bit E4M3
+ *                                     codes (not on the pages: a storage
+ *                                     variant).
+ *   attn_decode_paged_noalloc         the decode with a fixed scratch array
+ *                                     instead of a workspace.
+ *   attn_kv_append, attn_kv_append_fp8  write new tokens' K/V into the cache.
+ *   attn_page_pool_*                  a host-side page allocator and the page
+ *                                     tables it uploads.
+ *
  * Conventions shared by every entry point
  * ---------------------------------------
  * - Pointers named q, k, v, out, k_pool, v_pool, page_table, seq_lens and
