@@ -42,11 +42,28 @@ def _check(name, st):
 
 
 def _need_cuda(*ts):
+    dev = None
     for t in ts:
-        if t is not None and not t.is_cuda:
+        if t is None:
+            continue
+        if not t.is_cuda:
             raise ValueError("tensors must be CUDA tensors on the current device")
-        if t is not None and not t.is_contiguous():
+        if dev is None:
+            dev = torch.cuda.current_device()
+        if t.device.index != dev:
+            raise ValueError(f"tensor on {t.device}, but the current device is cuda:{dev}")
+        if not t.is_contiguous():
             raise ValueError("tensors must be contiguous")
+
+
+def _expect(t, name, shape, dtype):
+    """Host-side check that a tensor argument has the layout the C ABI will assume."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
 
 
 def attn_status_string(status: int) -> str:
@@ -62,8 +79,11 @@ def _prefill(name, dtype, q, k, v, causal, window, scale, out, stream):
         raise ValueError(f"{name} expects {dtype} q, k, v")
     B, Hq, Sq, D = q.shape
     _, Hkv, Skv, _ = k.shape
+    _expect(k, "k", (B, Hkv, Skv, D), dtype)
+    _expect(v, "v", (B, Hkv, Skv, D), dtype)
     if out is None:
         out = torch.empty_like(q)
+    _expect(out, "out", q.shape, dtype)
     _need_cuda(q, k, v, out)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
@@ -88,10 +108,14 @@ def _prefill_lse(name, dtype, q, k, v, causal, window, scale, out, lse, stream):
         raise ValueError(f"{name} expects {dtype} q, k, v")
     B, Hq, Sq, D = q.shape
     _, Hkv, Skv, _ = k.shape
+    _expect(k, "k", (B, Hkv, Skv, D), dtype)
+    _expect(v, "v", (B, Hkv, Skv, D), dtype)
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    _expect(out, "out", q.shape, dtype)
+    _expect(lse, "lse", (B, Hq, Sq), torch.float32)
     _need_cuda(q, k, v, out, lse)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
@@ -120,10 +144,17 @@ def attn_prefill_paged(q, k_pool, v_pool, page_table, seq_lens, *, max_seq_len, 
     B, Hq, Sq, D = q.shape
     num_pages, Hkv, page_size, _ = k_pool.shape
     max_pages = page_table.shape[1]
+    _expect(q, "q", (B, Hq, Sq, D), torch.bfloat16)
+    _expect(k_pool, "k_pool", (num_pages, Hkv, page_size, D), torch.bfloat16)
+    _expect(v_pool, "v_pool", (num_pages, Hkv, page_size, D), torch.bfloat16)
+    _expect(page_table, "page_table", (B, max_pages), torch.int32)
+    _expect(seq_lens, "seq_lens", (B,), torch.int32)
     if out is None:
         out = torch.empty_like(q)
     if lse is None and want_lse:
         lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    _expect(out, "out", q.shape, torch.bfloat16)
+    _expect(lse, "lse", (B, Hq, Sq), torch.float32)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     _need_cuda(q, k_pool, v_pool, page_table, seq_lens, out, lse)
@@ -134,6 +165,18 @@ def attn_prefill_paged(q, k_pool, v_pool, page_table, seq_lens, *, max_seq_len, 
         num_pages, max_pages, int(max_seq_len), float(scale), int(bool(causal)), int(window), _ptr(out), _ptr(lse),
         _stream(stream)))
     return (out, lse) if lse is not None else out
+
+
+def _check_decode_args(q, k_pool, v_pool, page_table, seq_lens, pool_dtype):
+    if q.dim() != 3 or k_pool.dim() != 4 or page_table.dim() != 2:
+        raise ValueError("q must be [N,Hq,D], the pools [num_pages,Hkv,page_size,D], page_table [N,max_pages]")
+    N, Hq, D = q.shape
+    num_pages, Hkv, page_size, _ = k_pool.shape
+    _expect(q, "q", (N, Hq, D), torch.bfloat16)
+    _expect(k_pool, "k_pool", (num_pages, Hkv, page_size, D), pool_dtype)
+    _expect(v_pool, "v_pool", (num_pages, Hkv, page_size, D), pool_dtype)
+    _expect(page_table, "page_table", (N, page_table.shape[1]), torch.int32)
+    _expect(seq_lens, "seq_lens", (N,), torch.int32)
 
 
 def attn_decode_paged_workspace_size(N, Hq, D, max_seq_len, page_size) -> int:
@@ -147,8 +190,10 @@ def attn_decode_paged(q, k_pool, v_pool, page_table, seq_lens, *, max_seq_len, s
     N, Hq, D = q.shape
     num_pages, Hkv, page_size, _ = k_pool.shape
     max_pages = page_table.shape[1]
+    _check_decode_args(q, k_pool, v_pool, page_table, seq_lens, torch.bfloat16)
     if out is None:
         out = torch.empty_like(q)
+    _expect(out, "out", q.shape, torch.bfloat16)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     need = attn_decode_paged_workspace_size(N, Hq, D, max_seq_len, page_size)
@@ -171,10 +216,10 @@ def attn_decode_paged_fp8(q, k_pool, v_pool, page_table, seq_lens, *, max_seq_le
     N, Hq, D = q.shape
     num_pages, Hkv, page_size, _ = k_pool.shape
     max_pages = page_table.shape[1]
-    if k_pool.dtype != torch.uint8 or v_pool.dtype != torch.uint8:
-        raise ValueError("k_pool and v_pool must hold uint8 E4M3 codes")
+    _check_decode_args(q, k_pool, v_pool, page_table, seq_lens, torch.uint8)
     if out is None:
         out = torch.empty_like(q)
+    _expect(out, "out", q.shape, torch.bfloat16)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     need = attn_decode_paged_workspace_size(N, Hq, D, max_seq_len, page_size)
@@ -200,8 +245,10 @@ def attn_decode_paged_noalloc(q, k_pool, v_pool, page_table, seq_lens, *, max_se
     N, Hq, D = q.shape
     num_pages, Hkv, page_size, _ = k_pool.shape
     max_pages = page_table.shape[1]
+    _check_decode_args(q, k_pool, v_pool, page_table, seq_lens, torch.bfloat16)
     if out is None:
         out = torch.empty_like(q)
+    _expect(out, "out", q.shape, torch.bfloat16)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     _need_cuda(q, k_pool, v_pool, page_table, seq_lens, out)
@@ -229,6 +276,8 @@ def attn_kv_append(k_new, v_new, k_pool, v_pool, page_table, seq_lens, *, stream
     if k_new.dtype != torch.bfloat16 or v_new.dtype != torch.bfloat16 or k_pool.dtype != torch.bfloat16 \
             or v_pool.dtype != torch.bfloat16:
         raise ValueError("k_new, v_new and the pools must be bfloat16")
+    _expect(page_table, "page_table", (B, page_table.shape[1]), torch.int32)
+    _expect(seq_lens, "seq_lens", (B,), torch.int32)
     _need_cuda(k_new, v_new, k_pool, v_pool, page_table, seq_lens)
     if page_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
         raise ValueError("page_table and seq_lens must be int32")
@@ -249,6 +298,8 @@ def attn_kv_append_fp8(k_new, v_new, k_pool, v_pool, page_table, seq_lens, *, k_
         raise ValueError("k_new and v_new must be bfloat16")
     if k_pool.dtype != torch.uint8 or v_pool.dtype != torch.uint8:
         raise ValueError("the pools must hold uint8 E4M3 codes")
+    _expect(page_table, "page_table", (B, page_table.shape[1]), torch.int32)
+    _expect(seq_lens, "seq_lens", (B,), torch.int32)
     _need_cuda(k_new, v_new, k_pool, v_pool, page_table, seq_lens)
     if page_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
         raise ValueError("page_table and seq_lens must be int32")
