@@ -330,7 +330,7 @@ def run_ours(args, rank, world, local_rank):
                          "kernel": "prefill_tc_kernel<64, false>", "peak_kind": f"bf16 burst, {peak_kind}"},
             "roofline_decode": {"bound": "hbm", "achieved": round(ach_d, 1), "peak": peak_h, "unit": "GB/s",
                                 "frac": round(ach_d / peak_h, 4), "traffic": traffic_d,
-                                "kernel": "decode_split_kernel<128,4> + decode_combine_kernel<128>",
+                                "kernel": "decode_split_kernel<128,4,false> + decode_combine_kernel<128>",
                                 "peak_kind": f"HBM copy, {peak_kind}"},
             "decode": {"value": round(job_rate(d_bytes, world, dec_ms) / 1e9, 1), "unit": "GB/s",
                        "ms": round(dec_ms, 5)},
