@@ -493,8 +493,16 @@ template <int D, int G, bool FP8>
 cudaError_t launch_split(const DecodeParams& p, int N, cudaStream_t stream) {
   const size_t smem = sizeof(SplitSmem<D, G, FP8>) + 1024;
   auto kern = decode_split_kernel<D, G, FP8>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
+  // the shared-memory limit is set once per device (a runtime call per launch costs host time)
+  constexpr int kMaxDevices = 64;
+  static int ready[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (__atomic_load_n(&ready[dev], __ATOMIC_ACQUIRE) != 1) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    __atomic_store_n(&ready[dev], 1, __ATOMIC_RELEASE);
+  }
   dim3 grid(p.max_splits, p.Hkv, N);
   kern<<<grid, kWarps * 32, smem, stream>>>(p);
   return cudaGetLastError();

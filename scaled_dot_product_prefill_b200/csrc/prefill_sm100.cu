@@ -776,19 +776,37 @@ int sm_count() {
   return cache[dev];
 }
 
+// One-time set-up of a kernel on the current device: its shared-memory limit,
+// and the check that setmaxnreg.inc can be honoured (it waits until the
+// block's own registers cover the request, so a build whose launch
+// allocation could not is refused).  Done once per device; later calls skip
+// the runtime queries, which cost more host time than the launch itself.
+template <int D, bool PAGED>
+cudaError_t prepare_kernel() {
+  constexpr int kMaxDevices = 64;
+  static int ready[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (__atomic_load_n(&ready[dev], __ATOMIC_ACQUIRE) == 1) return cudaSuccess;
+  auto kern = prefill_tc_kernel<D, PAGED>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(Cfg<D>::SMEM));
+  if (e != cudaSuccess) return e;
+  cudaFuncAttributes fa{};
+  e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs * kThreads < 128 * (2 * kSoftmaxRegs + kProducerRegs)) return cudaErrorInvalidConfiguration;
+  __atomic_store_n(&ready[dev], 1, __ATOMIC_RELEASE);
+  return cudaSuccess;
+}
+
 template <int D, bool PAGED>
 cudaError_t launch_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const Params& p,
                      cudaStream_t stream) {
   auto kern = prefill_tc_kernel<D, PAGED>;
   const size_t smem = Cfg<D>::SMEM;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  cudaError_t e = prepare_kernel<D, PAGED>();
   if (e != cudaSuccess) return e;
-  // setmaxnreg.inc waits until the block's own registers can cover the request:
-  // refuse to launch a build whose allocation could not.
-  cudaFuncAttributes fa{};
-  e = cudaFuncGetAttributes(&fa, kern);
-  if (e != cudaSuccess) return e;
-  if (fa.numRegs * kThreads < 128 * (2 * kSoftmaxRegs + kProducerRegs)) return cudaErrorInvalidConfiguration;
   const int sms = sm_count();
   if (sms <= 0) return cudaErrorInvalidDevice;
   const unsigned grid = static_cast<unsigned>(min(p.n_items, sms));
