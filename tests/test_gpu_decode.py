@@ -111,3 +111,16 @@ def test_sequence_longer_than_hint_is_reported():
     api.attn_device_status(clear=True)
     run_decode(p, max_seq_len=300)
     assert api.attn_device_status(clear=True) == 5
+
+
+def test_long_context_decode_merges_more_than_32_splits():
+    """70k tokens at 512 keys per split: the combine walks its splits in several blocks of 32."""
+    p = inputs.paged_inputs(2, 8, 2, 128, 16, seed=77, seq_lens=[40000, 70001], spare_pages=4, poison=True)
+    out = run_decode(p)
+    assert api.attn_device_status(clear=True) == 0
+    ref = sdpa.decode_paged(p.q, p.k_pool, p.v_pool, p.page_table, p.seq_lens, 16, 1 / np.sqrt(128))
+    assert_parity(out, ref, "bf16", "long context")
+    # with a window the first split is not split 0
+    out_w = run_decode(p, window=30000)
+    ref_w = sdpa.decode_paged(p.q, p.k_pool, p.v_pool, p.page_table, p.seq_lens, 16, 1 / np.sqrt(128), 30000)
+    assert_parity(out_w, ref_w, "bf16", "long context, window")

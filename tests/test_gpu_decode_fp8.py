@@ -135,3 +135,12 @@ def test_fp8_cache_filled_by_the_append_decodes_like_the_oracle():
     V = fp8.dequantize(fp8.quantize(v_new, vs), vs)
     ref = sdpa.attention(p.q.double().numpy()[:, :, None, :], K, V, 1 / np.sqrt(D), causal=True)[:, :, 0]
     assert_parity(out, ref, "bf16", "fp8 cache from the append")
+
+
+def test_fp8_long_context_decode():
+    ks, vs = 0.02, 0.02
+    p = inputs.paged_inputs_fp8(2, 8, 2, 128, 16, seed=78, k_scale=ks, v_scale=vs, seq_lens=[33333, 50000],
+                                poison=True)
+    out = run_fp8(p, ks, vs)
+    assert api.attn_device_status(clear=True) == 0
+    assert_parity(out, oracle_fp8(p, ks, vs, 1 / np.sqrt(128), 0), "bf16", "fp8 long context")

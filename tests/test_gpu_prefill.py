@@ -187,3 +187,17 @@ def test_lse_merges_two_key_halves_into_the_full_result():
     w1, w2 = torch.exp(l1 - m)[..., None], torch.exp(l2 - m)[..., None]
     merged = (w1 * o1.float() + w2 * o2.float()) / (w1 + w2)
     assert (merged - full.float()).abs().max().item() <= 2e-2
+
+
+@pytest.mark.parametrize("D,window", [(64, 0), (64, 3000), (128, 0)])
+def test_long_head_dim_64_and_128_sequences_on_sampled_rows(D, window):
+    """16k-token causal prefill at D = 64 (the separate-P pipeline over 128 key tiles per row block)."""
+    B, Hq, Hkv, S = 1, 4, 2, 16384
+    inp = inputs.prefill_inputs(B, Hq, Hkv, S, S, D, seed=91 + D + window)
+    out = run_prefill(inp, True, window).cpu()
+    rng = np.random.default_rng(D)
+    for h in range(Hq):
+        rows = sampled_rows(S, rng, n=24)
+        ref = sdpa.attention_rows(inp.q[0, h, rows], inp.k[0, h // 2], inp.v[0, h // 2], rows, S, 1 / np.sqrt(D),
+                                  True, window)
+        assert_parity(out[0, h, rows], ref, "bf16", f"S=16k D={D} W={window} h={h}")

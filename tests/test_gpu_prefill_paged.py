@@ -105,3 +105,16 @@ def test_paged_prefill_never_reads_entries_past_the_last_page():
     assert api.attn_device_status(clear=True) == 0
     ref, _ = oracle_paged_prefill(q, p, 1 / np.sqrt(128), False, 0)
     assert_parity(out, ref, "bf16", "junk past the last page")
+
+
+def test_paged_prefill_chunk_at_the_end_of_a_long_cache():
+    """A 512-token chunk whose cache holds 20k tokens in 64-token pages."""
+    L, Sq = 20000, 512
+    p = inputs.paged_inputs(1, 8, 2, 128, 64, seed=13, seq_lens=[L], spare_pages=3, poison=True)
+    q = inputs.normal((1, 8, Sq, 128), seed=14)
+    out = api.attn_prefill_paged(q.cuda(), p.k_pool.cuda(), p.v_pool.cuda(), p.page_table.cuda(), p.seq_lens.cuda(),
+                                 max_seq_len=L, causal=True)
+    torch.cuda.synchronize()
+    assert api.attn_device_status(clear=True) == 0
+    ref, _ = oracle_paged_prefill(q, p, 1 / np.sqrt(128), True, 0)
+    assert_parity(out, ref, "bf16", "20k cache, 512-token chunk")
