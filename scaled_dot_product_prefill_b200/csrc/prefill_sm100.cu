@@ -46,22 +46,12 @@ namespace attn {
 namespace {
 
 constexpr int BM = 128;          // query rows per tile
-constexpr int BN = 128;          // keys per tile
 constexpr int NQ = 2;            // query tiles per work item
-constexpr int kThreads = 384;    // 12 warps = 3 warpgroups
 constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;
-// Register split (setmaxnreg works per warpgroup): the two softmax groups hold
-// a 128-column score row each and get kSoftmaxRegs; the producer group (TMA
-// and MMA warps, two idle warps) gets kProducerRegs.  The split must fit the
-// launch allocation: 128 * (2 * kSoftmaxRegs + kProducerRegs) <= kThreads *
-// regs-per-thread at launch, which the host checks before every launch.
 #ifndef ATTN_PREFILL_TURNS
 #define ATTN_PREFILL_TURNS 0
 #endif
-constexpr int kSoftmaxRegs = 208;
-constexpr int kProducerRegs = 88;
-constexpr uint32_t kTmemCols = 512;
 constexpr float kTau = 8.0f;     // lazy-rescale threshold, log2 units
 // Of every 16 score pairs of a row, how many take exp2 on the FMA pipe
 // (exp2_fma2) instead of the MUFU unit, which is the bottleneck of the softmax.
@@ -70,28 +60,54 @@ constexpr float kTau = 8.0f;     // lazy-rescale threshold, log2 units
 #endif
 constexpr int kEmuPer16 = ATTN_EXP_EMU;
 
-template <int D>
+// D=64 layouts: 0 = one CTA per SM, 128-key tiles and P buffers of their own
+// (below); 1 = two CTAs per SM, each with 64-key tiles, P over S and half of
+// tensor memory, so that an SM runs four softmax chains instead of two.
+#ifndef ATTN_D64_VARIANT
+#define ATTN_D64_VARIANT 0
+#endif
+
+template <int D, int V = 0>
 struct Cfg {
+  static_assert(V == 0 || D == 64, "the two-CTA layout is for D = 64");
+  static constexpr int BN = (V == 1) ? 64 : 128;      // keys per tile
+  static constexpr int MINB = (V == 1) ? 2 : 1;       // CTAs per SM
+  static constexpr uint32_t TMEM_COLS = (V == 1) ? 256 : 512;
+  // V = 0: 12 warps (3 warpgroups) and a register split (setmaxnreg works per
+  // warpgroup): the two softmax groups hold a 128-column score row each; the
+  // producer group (TMA and MMA warps, two idle warps) gets the rest.
+  // 128 * (2 * SOFTMAX_REGS + PRODUCER_REGS) must fit the launch allocation
+  // (threads * registers per thread), which the host checks before the first
+  // launch.  V = 1: 10 warps (8 softmax, TMA, MMA) with about 100 registers
+  // each and no split.
+  static constexpr int THREADS = (V == 1) ? 320 : 384;
+  static constexpr bool SPLIT_REGS = (V == 0);
+  static constexpr int SOFTMAX_REGS = 208;
+  static constexpr int PRODUCER_REGS = 88;
   static constexpr int KATOMS = D / 64;               // 64-column (128-byte) swizzle atoms
   static constexpr int TILE_BYTES = BN * D * 2;       // one K or V tile
   static constexpr int Q_BYTES = BM * D * 2;          // one query tile
-  static constexpr int QBUF = (D == 128) ? 1 : 2;     // query buffers (items in flight)
+  static constexpr int QBUF = (D == 128 || V == 1) ? 1 : 2;   // query buffers (items in flight)
   static constexpr int STAGES = (D == 128) ? 4 : 6;   // ring slots; K and V tiles alternate
   // D = 64 leaves room in tensor memory for P buffers of their own (SEP_P):
   // S_i [128 i, +128), P_i [256 + 64 i, +64), O_i [384 + 64 i, +64).  The
   // softmax then releases S_i as soon as it has loaded it, and S_i(j+1) is
   // computed while the softmax of tile j is still running.  D = 128 has no
   // room: P_i is written over the first 64 columns of S_i, O_i [256 + 128 i, +128).
-  static constexpr bool SEP_P = (D == 64);
+  static constexpr bool SEP_P = (D == 64 && V == 0);
+  // O_i is rescaled after the exponentials (when its score registers are
+  // free) with separate P buffers, and in the small-register layout.
+  static constexpr bool LATE_RESCALE = SEP_P || V == 1;
   // TURNS: the two softmax groups take turns at the exponentials, so that one
   // group's exponentials run at the full MUFU rate while the other loads S,
   // takes its row max and stores P (ATTN_PREFILL_TURNS: 0 never, 1 at D = 64,
   // 2 always).
   static constexpr bool TURNS = (ATTN_PREFILL_TURNS == 2) || (ATTN_PREFILL_TURNS == 1 && D == 64);
-  static constexpr uint32_t S_COL = 0;                // + 128 * i
-  static constexpr uint32_t P_COL = SEP_P ? 256 : 0;  // + (SEP_P ? 64 : 128) * i
-  static constexpr uint32_t P_STRIDE = SEP_P ? 64 : 128;
-  static constexpr uint32_t O_COL = SEP_P ? 384 : 256;  // + D * i
+  // V = 1: S_i [64 i, +64) with P_i over its first 32 columns, O_i [128 + 64 i, +64).
+  static constexpr uint32_t S_COL = 0;                // + BN * i
+  static constexpr uint32_t P_COL = SEP_P ? 256 : 0;  // + P_STRIDE * i
+  static constexpr uint32_t P_STRIDE = SEP_P ? 64 : BN;
+  static constexpr uint32_t O_COL = SEP_P ? 384 : NQ * BN;  // + D * i
   static constexpr size_t SMEM = 1024 /*align*/ + QBUF * NQ * Q_BYTES + STAGES * TILE_BYTES + 256;
 };
 
@@ -122,7 +138,7 @@ __device__ __forceinline__ int item_index(const Params& p, int r) {
   return k < p.n_items ? k : -1;
 }
 
-template <bool PAGED>
+template <int BN, bool PAGED>
 __device__ __forceinline__ Item make_item(const Params& p, int k) {
   Item it;
   const int BH = p.B * p.Hq;
@@ -174,6 +190,7 @@ __device__ __forceinline__ bool active(const Item& it, int i, int j) { return j 
 
 // True if every (row, key) pair of query rows [r0, r0+BM) x key tile j is visible
 // (skv keys in the sequence).
+template <int BN>
 __device__ __forceinline__ bool tile_unmasked(const Params& p, int skv, int r0, int j) {
   const int off = skv - p.Sq;
   const int k0 = j * BN, k1 = j * BN + BN - 1;
@@ -187,11 +204,12 @@ __device__ __forceinline__ bool tile_unmasked(const Params& p, int skv, int r0, 
 // PAGED selects K/V through a page table (chunked prefill over a paged cache)
 // instead of dense [B, Hkv, Skv, D] tensors; the dense kernel carries none of
 // the paged code.
-template <int D, bool PAGED>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int D, bool PAGED, int V>
+__global__ void __launch_bounds__(Cfg<D, V>::THREADS, Cfg<D, V>::MINB)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_v, const Params p) {
-  using C = Cfg<D>;
+  using C = Cfg<D, V>;
+  constexpr int BN = C::BN;
   constexpr int STAGES = C::STAGES, QBUF = C::QBUF;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -236,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -246,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp >= 8) {
    // ------------------------------------------------------------ producer warpgroup
-   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
+   if constexpr (C::SPLIT_REGS) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::PRODUCER_REGS));
    if (warp == kTmaWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -258,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int r = 0; r < n_rounds && ok; ++r) {
         const int k = item_index(p, r);
         if (k < 0) continue;
-        const Item it = make_item<PAGED>(p, k);
+        const Item it = make_item<BN, PAGED>(p, k);
         if (it.hi_all <= it.lo_all) continue;
         const int qb = qn % QBUF;
         if (qn >= QBUF && !(ok = mbar_wait(&q_empty[qb], ((qn / QBUF) - 1) & 1, abort_flag, p.err))) break;
@@ -345,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
 
       auto issue_s = [&](int i, int qb, int st) {  // S_i = Q_i K^T from ring slot st
-        const uint32_t d_tmem = tmem + C::S_COL + 128 * i;
+        const uint32_t d_tmem = tmem + C::S_COL + BN * i;
         const uint32_t a_lo = q_lo0 + (((qb * NQ + i) * C::Q_BYTES) >> 4);
         const uint32_t b_lo = k_lo0 + ((st * C::TILE_BYTES) >> 4);
 #pragma unroll
@@ -390,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int r = 0; r < n_rounds && ok; ++r) {
           const int k = item_index(p, r);
           if (k < 0) continue;
-          const Item it = make_item<PAGED>(p, k);
+          const Item it = make_item<BN, PAGED>(p, k);
           if (it.hi_all <= it.lo_all) continue;
           const int qb = qn % QBUF;
           if (!(ok = mbar_wait(&q_full[qb], (qn / QBUF) & 1, abort_flag, p.err))) break;
@@ -457,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int r = 0; r < n_rounds && ok; ++r) {
           const int k = item_index(p, r);
           if (k < 0) continue;
-          const Item it = make_item<PAGED>(p, k);
+          const Item it = make_item<BN, PAGED>(p, k);
           if (it.hi_all <= it.lo_all) continue;
           const int qb = qn % QBUF;
           if (!(ok = mbar_wait(&q_full[qb], (qn / QBUF) & 1, abort_flag, p.err))) break;
@@ -514,12 +532,12 @@ __global__ void __launch_bounds__(kThreads, 1)
    }
   } else {
     // ------------------------------------------------------------ softmax groups
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+    if constexpr (C::SPLIT_REGS) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::SOFTMAX_REGS));
     const int i = warp >> 2;                 // query tile
     const int wq = warp & 3;                 // lane quarter of tensor memory
     const int rl = wq * 32 + lane;           // row within the tile
     const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t s_tmem = tmem + lane_bits + C::S_COL + 128 * i;
+    const uint32_t s_tmem = tmem + lane_bits + C::S_COL + BN * i;
     const uint32_t p_tmem = tmem + lane_bits + C::P_COL + C::P_STRIDE * i;
     const uint32_t o_tmem = tmem + lane_bits + C::O_COL + D * i;
     const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
@@ -563,7 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int rr = 0; rr < n_rounds && ok; ++rr) {
       const int k = item_index(p, rr);
       if (k < 0) continue;
-      const Item it = make_item<PAGED>(p, k);
+      const Item it = make_item<BN, PAGED>(p, k);
       const int my_lo = (i == 0) ? it.lo[0] : it.lo[1];
       const int my_hi = (i == 0) ? it.hi[0] : it.hi[1];
       if constexpr (C::TURNS) {
@@ -609,15 +627,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
           mbar_arrive(&s_free[i]);
         }
-        if (!tile_unmasked(p, skv, r0, j)) {
+        if (!tile_unmasked<BN>(p, skv, r0, j)) {
           const int c_lo = key_lo - j * BN, c_hi = key_hi - j * BN;
 #pragma unroll
           for (int c = 0; c < BN; ++c) s[c] = (c >= c_lo && c <= c_hi) ? s[c] : -INFINITY;
         }
         // row maximum: four independent chains of three-input max
-        float mc[4] = {s[0], s[1], s[2], s[3]};
+        // (columns 0-7 start the chains, then 8 columns per step: exactly s[0, BN))
+        float mc[4];
 #pragma unroll
-        for (int c = 4; c < BN; c += 8)
+        for (int q = 0; q < 4; ++q) mc[q] = fmaxf(s[2 * q], s[2 * q + 1]);
+#pragma unroll
+        for (int c = 8; c < BN; c += 8)
 #pragma unroll
           for (int q = 0; q < 4; ++q) mc[q] = fmax3(mc[q], s[c + 2 * q], s[c + 2 * q + 1]);
         const float mx = fmaxf(fmax3(mc[0], mc[1], mc[2]), mc[3]);
@@ -628,7 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           l *= alpha;
           m_ref = m_tile;
         }
-        if constexpr (!C::SEP_P) rescale_o(j > my_lo, alpha);   // O_i is current: S_i(j) covers P_i V(j-1)
+        if constexpr (!C::LATE_RESCALE) rescale_o(j > my_lo, alpha);   // O_i is current: S_i(j) covers P_i V(j-1)
         if constexpr (C::TURNS) {
           if (!(ok = take_turn())) break;
         }
@@ -672,7 +693,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
           }
         }
-        if constexpr (C::SEP_P) rescale_o(j > my_lo, alpha);
+        if constexpr (C::LATE_RESCALE) rescale_o(j > my_lo, alpha);
 #pragma unroll
         for (int c = 0; c < BN / 64; ++c) tmem_st32(p_tmem + 32 * c, pk + 32 * c);
         tmem_wait_st();
@@ -724,7 +745,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
@@ -781,36 +802,38 @@ int sm_count() {
 // block's own registers cover the request, so a build whose launch
 // allocation could not is refused).  Done once per device; later calls skip
 // the runtime queries, which cost more host time than the launch itself.
-template <int D, bool PAGED>
+template <int D, bool PAGED, int V>
 cudaError_t prepare_kernel() {
+  using C = Cfg<D, V>;
   constexpr int kMaxDevices = 64;
   static int ready[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   if (__atomic_load_n(&ready[dev], __ATOMIC_ACQUIRE) == 1) return cudaSuccess;
-  auto kern = prefill_tc_kernel<D, PAGED>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(Cfg<D>::SMEM));
+  auto kern = prefill_tc_kernel<D, PAGED, V>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM));
   if (e != cudaSuccess) return e;
   cudaFuncAttributes fa{};
   e = cudaFuncGetAttributes(&fa, kern);
   if (e != cudaSuccess) return e;
-  if (fa.numRegs * kThreads < 128 * (2 * kSoftmaxRegs + kProducerRegs)) return cudaErrorInvalidConfiguration;
+  if (C::SPLIT_REGS && fa.numRegs * C::THREADS < 128 * (2 * C::SOFTMAX_REGS + C::PRODUCER_REGS))
+    return cudaErrorInvalidConfiguration;
   __atomic_store_n(&ready[dev], 1, __ATOMIC_RELEASE);
   return cudaSuccess;
 }
 
-template <int D, bool PAGED>
+template <int D, bool PAGED, int V>
 cudaError_t launch_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const Params& p,
                      cudaStream_t stream) {
-  auto kern = prefill_tc_kernel<D, PAGED>;
-  const size_t smem = Cfg<D>::SMEM;
-  cudaError_t e = prepare_kernel<D, PAGED>();
+  using C = Cfg<D, V>;
+  auto kern = prefill_tc_kernel<D, PAGED, V>;
+  const size_t smem = C::SMEM;
+  cudaError_t e = prepare_kernel<D, PAGED, V>();
   if (e != cudaSuccess) return e;
   const int sms = sm_count();
   if (sms <= 0) return cudaErrorInvalidDevice;
-  const unsigned grid = static_cast<unsigned>(min(p.n_items, sms));
-  kern<<<grid, kThreads, smem, stream>>>(mq, mk, mv, p);
+  const unsigned grid = static_cast<unsigned>(min(p.n_items, sms * C::MINB));
+  kern<<<grid, C::THREADS, smem, stream>>>(mq, mk, mv, p);
   return cudaGetLastError();
 }
 
@@ -819,8 +842,11 @@ cudaError_t launch_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
 cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
                               int Hkv, int Sq, int Skv, int D, float scale, int causal, int window, unsigned int* err,
                               cudaStream_t stream) {
+  constexpr int V64 = ATTN_D64_VARIANT;
+  const int bn = (D == 64) ? Cfg<64, V64>::BN : Cfg<128, 0>::BN;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, D, Sq, B * Hq) || !make_map(&mk, k, D, Skv, B * Hkv) || !make_map(&mv, v, D, Skv, B * Hkv))
+  if (!make_map(&mq, q, D, Sq, B * Hq) || !make_map(&mk, k, D, Skv, B * Hkv, bn) ||
+      !make_map(&mv, v, D, Skv, B * Hkv, bn))
     return cudaErrorInvalidValue;
   Params p{};
   p.B = B;
@@ -838,14 +864,16 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, void*
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
   p.err = err;
-  return D == 64 ? launch_d<64, false>(mq, mk, mv, p, stream) : launch_d<128, false>(mq, mk, mv, p, stream);
+  return D == 64 ? launch_d<64, false, V64>(mq, mk, mv, p, stream) : launch_d<128, false, 0>(mq, mk, mv, p, stream);
 }
 
 cudaError_t launch_prefill_tc_paged(const void* q, const void* k_pool, const void* v_pool, const int32_t* page_table,
                                     const int32_t* seq_lens, int page_size, int B, int Hq, int Hkv, int Sq, int D,
                                     int num_pages, int max_pages, int max_seq_len, float scale, int causal,
                                     int window, void* out, float* lse, unsigned int* err, cudaStream_t stream) {
-  const int box_rows = page_size < BM ? page_size : BM;
+  constexpr int V64 = ATTN_D64_VARIANT;
+  const int bn = (D == 64) ? Cfg<64, V64>::BN : Cfg<128, 0>::BN;
+  const int box_rows = page_size < bn ? page_size : bn;
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, q, D, Sq, B * Hq) || !make_map(&mk, k_pool, D, page_size, num_pages * Hkv, box_rows) ||
       !make_map(&mv, v_pool, D, page_size, num_pages * Hkv, box_rows))
@@ -872,7 +900,7 @@ cudaError_t launch_prefill_tc_paged(const void* q, const void* k_pool, const voi
   p.box_rows = box_rows;
   p.max_pages = max_pages;
   p.num_pages = num_pages;
-  return D == 64 ? launch_d<64, true>(mq, mk, mv, p, stream) : launch_d<128, true>(mq, mk, mv, p, stream);
+  return D == 64 ? launch_d<64, true, V64>(mq, mk, mv, p, stream) : launch_d<128, true, 0>(mq, mk, mv, p, stream);
 }
 
 }  // namespace attn
