@@ -327,7 +327,7 @@ def run_ours(args, rank, world, local_rank):
             },
             "roofline": {"bound": "tensor", "achieved": round(ach_t, 2), "peak": peak_t, "unit": "TFLOP/s",
                          "frac": round(ach_t / peak_t, 4), "traffic": traffic,
-                         "kernel": "prefill_tc_kernel<64, false>", "peak_kind": f"bf16 burst, {peak_kind}"},
+                         "kernel": "prefill_tc_kernel<64, false, 0>", "peak_kind": f"bf16 burst, {peak_kind}"},
             "roofline_decode": {"bound": "hbm", "achieved": round(ach_d, 1), "peak": peak_h, "unit": "GB/s",
                                 "frac": round(ach_d / peak_h, 4), "traffic": traffic_d,
                                 "kernel": "decode_split_kernel<128,4,false> + decode_combine_kernel<128>",
