@@ -66,10 +66,15 @@ constexpr int kEmuPer16 = ATTN_EXP_EMU;
 #ifndef ATTN_D64_VARIANT
 #define ATTN_D64_VARIANT 0
 #endif
+// D=128 layouts: 0 = P written over S in tensor memory; 2 = P in shared memory
+// (a 3-slot K/V ring makes room), so that S_i(j+1) need not wait for P_i V(j).
+#ifndef ATTN_D128_VARIANT
+#define ATTN_D128_VARIANT 0
+#endif
 
 template <int D, int V = 0>
 struct Cfg {
-  static_assert(V == 0 || D == 64, "the two-CTA layout is for D = 64");
+  static_assert(V == 0 || (V == 1 && D == 64) || (V == 2 && D == 128), "layout variant");
   static constexpr int BN = (V == 1) ? 64 : 128;      // keys per tile
   static constexpr int MINB = (V == 1) ? 2 : 1;       // CTAs per SM
   static constexpr uint32_t TMEM_COLS = (V == 1) ? 256 : 512;
@@ -88,13 +93,15 @@ struct Cfg {
   static constexpr int TILE_BYTES = BN * D * 2;       // one K or V tile
   static constexpr int Q_BYTES = BM * D * 2;          // one query tile
   static constexpr int QBUF = (D == 128 || V == 1) ? 1 : 2;   // query buffers (items in flight)
-  static constexpr int STAGES = (D == 128) ? 4 : 6;   // ring slots; K and V tiles alternate
+  static constexpr int STAGES = (D == 128) ? (V == 2 ? 3 : 4) : 6;   // ring slots; K and V tiles alternate
   // D = 64 leaves room in tensor memory for P buffers of their own (SEP_P):
   // S_i [128 i, +128), P_i [256 + 64 i, +64), O_i [384 + 64 i, +64).  The
   // softmax then releases S_i as soon as it has loaded it, and S_i(j+1) is
   // computed while the softmax of tile j is still running.  D = 128 has no
   // room: P_i is written over the first 64 columns of S_i, O_i [256 + 128 i, +128).
-  static constexpr bool SEP_P = (D == 64 && V == 0);
+  static constexpr bool SEP_P = (D == 64 && V == 0) || V == 2;
+  static constexpr bool P_SMEM = (V == 2);            // P_i in shared memory, read by an SS-form P.V
+  static constexpr int P_BYTES = P_SMEM ? NQ * BM * BN * 2 : 0;
   // O_i is rescaled after the exponentials (when its score registers are
   // free) with separate P buffers, and in the small-register layout.
   static constexpr bool LATE_RESCALE = SEP_P || V == 1;
@@ -107,8 +114,8 @@ struct Cfg {
   static constexpr uint32_t S_COL = 0;                // + BN * i
   static constexpr uint32_t P_COL = SEP_P ? 256 : 0;  // + P_STRIDE * i
   static constexpr uint32_t P_STRIDE = SEP_P ? 64 : BN;
-  static constexpr uint32_t O_COL = SEP_P ? 384 : NQ * BN;  // + D * i
-  static constexpr size_t SMEM = 1024 /*align*/ + QBUF * NQ * Q_BYTES + STAGES * TILE_BYTES + 256;
+  static constexpr uint32_t O_COL = (SEP_P && !P_SMEM) ? 384 : NQ * BN;  // + D * i
+  static constexpr size_t SMEM = 1024 /*align*/ + QBUF * NQ * Q_BYTES + STAGES * TILE_BYTES + P_BYTES + 256;
 };
 
 struct Params {
@@ -216,7 +223,8 @@ __global__ void __launch_bounds__(Cfg<D, V>::THREADS, Cfg<D, V>::MINB)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = smem;                                   // [QBUF][NQ][KATOMS][BM rows x 128 B]
   uint8_t* sRing = smem + QBUF * NQ * C::Q_BYTES;       // [STAGES][KATOMS][BN rows x 128 B]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sRing + STAGES * C::TILE_BYTES);
+  uint8_t* sP = sRing + STAGES * C::TILE_BYTES;         // P_SMEM: [NQ][BN / 64][BM rows x 128 B]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + C::P_BYTES);
   uint64_t* q_full = bars;                              // QBUF
   uint64_t* q_empty = q_full + QBUF;                    // QBUF
   uint64_t* full = q_empty + QBUF;                      // STAGES
@@ -358,6 +366,7 @@ __global__ void __launch_bounds__(Cfg<D, V>::THREADS, Cfg<D, V>::MINB)
       const uint32_t q_lo0 = sw128_desc_lo(smem_u32(sQ), 16);
       const uint32_t k_lo0 = sw128_desc_lo(smem_u32(sRing), 16);
       const uint32_t v_lo0 = sw128_desc_lo(smem_u32(sRing), BN * 128);
+      const uint32_t p_lo0 = sw128_desc_lo(smem_u32(sP), 16);   // P_SMEM only
       int n = 0, qn = 0;
       int ts[NQ] = {0, 0};
       bool ok = true;
@@ -450,13 +459,23 @@ __global__ void __launch_bounds__(Cfg<D, V>::THREADS, Cfg<D, V>::MINB)
               tc_fence_after();
               ++ts[i];
               const uint32_t o_tmem = tmem + C::O_COL + D * i;
-              const uint32_t p_tmem = tmem + C::P_COL + C::P_STRIDE * i;
               const uint32_t vb_lo = v_lo0 + ((stV * C::TILE_BYTES) >> 4);
               const uint32_t acc0 = (j > it.lo[i]) ? 1u : 0u;
+              if constexpr (C::P_SMEM) {   // A = P_i, K-major in shared memory like a Q tile
+                const uint32_t pa_lo = p_lo0 + ((i * BM * BN * 2) >> 4);
 #pragma unroll
-              for (int kk = 0; kk < BN / 16; ++kk)
-                mma_ts(o_tmem, p_tmem + kk * 8, desc64(vb_lo + ((kk * 16 * 128) >> 4), kHi), idesc_pv,
-                       kk > 0 ? 1u : acc0);
+                for (int kk = 0; kk < BN / 16; ++kk) {
+                  const uint32_t koff = ((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4;
+                  mma_ss(o_tmem, desc64(pa_lo + koff, kHi), desc64(vb_lo + ((kk * 16 * 128) >> 4), kHi), idesc_pv,
+                         kk > 0 ? 1u : acc0);
+                }
+              } else {
+                const uint32_t p_tmem = tmem + C::P_COL + C::P_STRIDE * i;
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk)
+                  mma_ts(o_tmem, p_tmem + kk * 8, desc64(vb_lo + ((kk * 16 * 128) >> 4), kHi), idesc_pv,
+                         kk > 0 ? 1u : acc0);
+              }
               mma_commit(&o_done[i]);   // P_i free again, O_i current
             }
             if (!ok) break;
@@ -694,9 +713,23 @@ __global__ void __launch_bounds__(Cfg<D, V>::THREADS, Cfg<D, V>::MINB)
           }
         }
         if constexpr (C::LATE_RESCALE) rescale_o(j > my_lo, alpha);
+        if constexpr (C::P_SMEM) {
+          // row rl of P_i in the 128-byte-swizzled K-major layout the MMA reads:
+          // 16-byte chunk c of a 128-byte row lands at chunk c ^ (row % 8)
+          const uint32_t prow = smem_u32(sP) + i * (BM * BN * 2) + rl * 128;
 #pragma unroll
-        for (int c = 0; c < BN / 64; ++c) tmem_st32(p_tmem + 32 * c, pk + 32 * c);
-        tmem_wait_st();
+          for (int ch = 0; ch < BN / 8; ++ch) {
+            const uint32_t addr = prow + (ch >> 3) * (BM * 128) + (((ch & 7) ^ (rl & 7)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * ch]),
+                         "r"(pk[4 * ch + 1]), "r"(pk[4 * ch + 2]), "r"(pk[4 * ch + 3])
+                         : "memory");
+          }
+          fence_proxy_async_smem();   // the MMA reads P through the async proxy
+        } else {
+#pragma unroll
+          for (int c = 0; c < BN / 64; ++c) tmem_st32(p_tmem + 32 * c, pk + 32 * c);
+          tmem_wait_st();
+        }
         tc_fence_before();
         mbar_arrive(&p_ready[i]);
       }
@@ -843,7 +876,7 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, void*
                               int Hkv, int Sq, int Skv, int D, float scale, int causal, int window, unsigned int* err,
                               cudaStream_t stream) {
   constexpr int V64 = ATTN_D64_VARIANT;
-  const int bn = (D == 64) ? Cfg<64, V64>::BN : Cfg<128, 0>::BN;
+  const int bn = (D == 64) ? Cfg<64, V64>::BN : Cfg<128, ATTN_D128_VARIANT>::BN;
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, q, D, Sq, B * Hq) || !make_map(&mk, k, D, Skv, B * Hkv, bn) ||
       !make_map(&mv, v, D, Skv, B * Hkv, bn))
@@ -864,7 +897,8 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, void*
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
   p.err = err;
-  return D == 64 ? launch_d<64, false, V64>(mq, mk, mv, p, stream) : launch_d<128, false, 0>(mq, mk, mv, p, stream);
+  return D == 64 ? launch_d<64, false, V64>(mq, mk, mv, p, stream)
+                 : launch_d<128, false, ATTN_D128_VARIANT>(mq, mk, mv, p, stream);
 }
 
 cudaError_t launch_prefill_tc_paged(const void* q, const void* k_pool, const void* v_pool, const int32_t* page_table,
@@ -872,7 +906,7 @@ cudaError_t launch_prefill_tc_paged(const void* q, const void* k_pool, const voi
                                     int num_pages, int max_pages, int max_seq_len, float scale, int causal,
                                     int window, void* out, float* lse, unsigned int* err, cudaStream_t stream) {
   constexpr int V64 = ATTN_D64_VARIANT;
-  const int bn = (D == 64) ? Cfg<64, V64>::BN : Cfg<128, 0>::BN;
+  const int bn = (D == 64) ? Cfg<64, V64>::BN : Cfg<128, ATTN_D128_VARIANT>::BN;
   const int box_rows = page_size < bn ? page_size : bn;
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, q, D, Sq, B * Hq) || !make_map(&mk, k_pool, D, page_size, num_pages * Hkv, box_rows) ||
@@ -900,7 +934,8 @@ cudaError_t launch_prefill_tc_paged(const void* q, const void* k_pool, const voi
   p.box_rows = box_rows;
   p.max_pages = max_pages;
   p.num_pages = num_pages;
-  return D == 64 ? launch_d<64, true, V64>(mq, mk, mv, p, stream) : launch_d<128, true, 0>(mq, mk, mv, p, stream);
+  return D == 64 ? launch_d<64, true, V64>(mq, mk, mv, p, stream)
+                 : launch_d<128, true, ATTN_D128_VARIANT>(mq, mk, mv, p, stream);
 }
 
 }  // namespace attn
