@@ -489,6 +489,55 @@ def other_workloads(dev, peaks):
     return res
 
 
+def profile_case(name, calls):
+    """Run one workload ``calls`` times and nothing else, for a profiler capture of its kernels.
+
+    ``name`` is a prefill workload of ``workloads.WORKLOADS``, ``paged_decode_gqa``, or
+    ``paged_decode_gqa_fp8`` (the same decode over an 8-bit cache).  Prints one line with the
+    mean CUDA-event time, which is not a benchmark number when taken under a profiler.
+    """
+    import torch
+
+    from scaled_dot_product_prefill_b200 import api
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    if name.startswith("paged_decode_gqa"):
+        spec = workloads.WORKLOADS["paged_decode_gqa"]
+        fp8 = name.endswith("_fp8")
+        if fp8:
+            pd = inputs.paged_inputs_fp8(spec.N, spec.Hq, spec.Hkv, spec.D, spec.page_size, spec.seed,
+                                         k_scale=1 / 64, v_scale=1 / 64, len_range=spec.len_range)
+        else:
+            pd = inputs.paged_inputs(spec.N, spec.Hq, spec.Hkv, spec.D, spec.page_size, spec.seed,
+                                     len_range=spec.len_range)
+        dq, kp, vp, pt, sl = (t.to(dev) for t in (pd.q, pd.k_pool, pd.v_pool, pd.page_table, pd.seq_lens))
+        ws = torch.empty(api.attn_decode_paged_workspace_size(spec.N, spec.Hq, spec.D, pd.max_seq_len,
+                                                              spec.page_size), dtype=torch.uint8, device=dev)
+        out = torch.empty_like(dq)
+        if fp8:
+            fn = lambda: api.attn_decode_paged_fp8(dq, kp, vp, pt, sl, max_seq_len=pd.max_seq_len, k_scale=1 / 64,
+                                                   v_scale=1 / 64, scale=spec.scale, workspace=ws, out=out)
+        else:
+            fn = lambda: api.attn_decode_paged(dq, kp, vp, pt, sl, max_seq_len=pd.max_seq_len, scale=spec.scale,
+                                               workspace=ws, out=out)
+    else:
+        spec = workloads.WORKLOADS[name]
+        pi = inputs.prefill_inputs(spec.B, spec.Hq, spec.Hkv, spec.Sq, spec.Skv, spec.D, spec.seed, spec.dtype)
+        q, k, v = pi.q.to(dev), pi.k.to(dev), pi.v.to(dev)
+        out = torch.empty_like(q)
+        call = api.attn_prefill if spec.dtype == "bf16" else api.attn_prefill_f32
+        fn = lambda: call(q, k, v, causal=spec.causal, window=spec.window, scale=spec.scale, out=out)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record()
+    for _ in range(calls):
+        fn()
+    ev[1].record()
+    torch.cuda.synchronize()
+    assert api.attn_device_status(clear=True) == 0
+    print(json.dumps({"profile_case": name, "calls": calls, "ms_per_call": ev[0].elapsed_time(ev[1]) / calls}))
+
+
 def reference_line(args, rank, world):
     """The float64 oracle on the host cores, on a bounded sample of the same workload."""
     if rank != 0:
@@ -518,12 +567,18 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--profile", default=None,
+                    help="run only this workload --steps times, for a profiler capture (prints no bench line)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", args.gpus if args.gpus == 1 else 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
     threads = cpu_threads()
     os.environ.setdefault("OMP_NUM_THREADS", str(threads))
+
+    if args.profile is not None:
+        profile_case(args.profile, max(1, args.steps))
+        return
 
     if args.impl == "reference":
         line = reference_line(args, rank, world)
