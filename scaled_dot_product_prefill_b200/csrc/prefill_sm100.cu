@@ -33,6 +33,16 @@
 // result stays exact.  Key tiles that the mask hides from every row of a
 // query tile are never loaded or multiplied; element masks are applied only
 // on tiles that straddle a mask edge.
+//
+// At D = 64 tensor memory has room for P buffers of their own (Cfg::SEP_P):
+// the softmax releases S_i as soon as it has loaded it, the MMA thread
+// computes S_i(j+1) while the exponentials of tile j run, and each P_i V_j
+// signals its own completion.  PAGED kernels read K/V through a page table
+// as page-sized TMA boxes.  Compile-time alternatives, measured and left
+// off: ATTN_D64_VARIANT=1 (two CTAs per SM over 64-key tiles),
+// ATTN_D128_VARIANT=2 (P in shared memory), ATTN_PREFILL_TURNS (the softmax
+// groups take turns at the exponentials), ATTN_EXP_EMU (part of the
+// exponentials on the FMA pipe).
 #include <cmath>
 #include <cstdint>
 #include <cuda.h>
