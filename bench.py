@@ -48,10 +48,20 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+def code_of(text):
+    """C++/CUDA source with comments removed and each line's whitespace trimmed (string literals kept)."""
+    import re
+
+    pattern = re.compile(r'//[^\n]*|/\*.*?\*/|"(?:\\.|[^"\\])*"', re.S)
+    text = pattern.sub(lambda m: m.group(0) if m.group(0).startswith('"') else " ", text)
+    return "\n".join(line.strip() for line in text.splitlines() if line.strip())
+
+
 def source_sha(name):
+    """First 16 hex digits of the sha256 of a kernel source's code (comments and layout ignored)."""
     p = os.path.join(ROOT, "scaled_dot_product_prefill_b200", "csrc", name)
-    with open(p, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    with open(p, encoding="utf-8") as f:
+        return hashlib.sha256(code_of(f.read()).encode()).hexdigest()[:16]
 
 
 def recorded_traffic(kernel, workload, src):
