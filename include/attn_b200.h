@@ -300,6 +300,18 @@ size_t attn_decode_paged_workspace_size(int N, int Hq, int D, int max_seq_len, i
 attn_status_t attn_device_status(int clear);
 
 /*
+ * attn_selftest_wait_timeout -- exercise the failure path of the kernels'
+ * bounded waits.  Launches one thread that waits, with the same wait the
+ * kernels use, for an mbarrier phase that nothing completes; after limit_ms
+ * milliseconds (1 to 1000) the wait gives up, records ATTN_ERR_TIMEOUT in
+ * the device error word and the kernel returns.  attn_device_status then
+ * reports ATTN_ERR_TIMEOUT, and the CUDA context stays usable.  A
+ * diagnostic with no counterpart in the pages.
+ * Errors: ATTN_ERR_INVALID_ARG (limit out of range), ATTN_ERR_CUDA.
+ */
+attn_status_t attn_selftest_wait_timeout(int limit_ms, attn_stream_t stream);
+
+/*
  * ---------------------------------------------------------------------------
  * Paged KV cache management: a host-side page pool and the append kernel.
  *

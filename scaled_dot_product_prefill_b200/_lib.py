@@ -28,6 +28,7 @@ PROTOTYPES = {
     "attn_decode_paged_noalloc": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 8 + [_c_float, _c_int, _vp, _vp]),
     "attn_decode_paged_workspace_size": (_c_size, [_c_int] * 5),
     "attn_device_status": (_c_int, [_c_int]),
+    "attn_selftest_wait_timeout": (_c_int, [_c_int, _vp]),
     "attn_kv_append": (_c_int, [_vp] * 6 + [_c_int] * 7 + [_vp]),
     "attn_kv_append_fp8": (_c_int, [_vp] * 6 + [_c_int] * 7 + [_c_float, _c_float, _vp]),
     "attn_page_pool_create": (_c_int, [_c_int] * 4 + [ctypes.POINTER(_vp)]),

@@ -17,7 +17,7 @@ __all__ = ["attn_prefill", "attn_prefill_f32", "attn_prefill_lse", "attn_prefill
            "attn_prefill_paged", "attn_decode_paged", "attn_decode_paged_noalloc",
            "attn_decode_paged_workspace_size", "attn_decode_paged_fp8", "attn_kv_append", "attn_kv_append_fp8",
            "PagePool",
-           "attn_device_status", "attn_status_string", "attn_version", "AttnError"]
+           "attn_device_status", "attn_selftest_wait_timeout", "attn_status_string", "attn_version", "AttnError"]
 
 
 def _stream(stream):
@@ -365,3 +365,8 @@ class PagePool:
         _need_cuda(page_table, seq_lens)
         _check("attn_page_pool_upload", self._lib.attn_page_pool_upload(
             self._h, _ptr(page_table), _ptr(seq_lens), _stream(stream)))
+
+
+def attn_selftest_wait_timeout(limit_ms=20, stream=None):
+    """Run a kernel whose bounded wait expires after limit_ms; attn_device_status() then reports a timeout."""
+    _check("attn_selftest_wait_timeout", _lib.load().attn_selftest_wait_timeout(int(limit_ms), _stream(stream)))

@@ -9,6 +9,7 @@
 
 #include "attn_b200.h"
 #include "common.cuh"
+#include "sm100_ptx.cuh"
 
 namespace attn {
 
@@ -311,6 +312,38 @@ attn_status_t attn_kv_append_fp8(const void* k_new, const void* v_new, uint8_t* 
                                  attn_stream_t stream) {
   return kv_append(k_new, v_new, k_pool, v_pool, page_table, seq_lens, page_size, B, Hkv, S_new, D, num_pages,
                    max_pages, stream, true, k_scale, v_scale);
+}
+
+}  // extern "C"
+
+namespace attn {
+namespace {
+
+// One thread waits, through the kernels' own bounded wait, for an mbarrier
+// phase that nothing completes; the wait gives up after limit_ns and records
+// a timeout in the error word, and the kernel returns normally.
+__global__ void timeout_selftest_kernel(unsigned int* err, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  abort_flag = 0;
+  mbar_wait_for(&bar, 0, &abort_flag, err, limit_ns);
+}
+
+}  // namespace
+}  // namespace attn
+
+extern "C" {
+
+attn_status_t attn_selftest_wait_timeout(int limit_ms, attn_stream_t stream) {
+  if (limit_ms < 1 || limit_ms > 1000) return ATTN_ERR_INVALID_ARG;
+  unsigned int* err = attn::device_error_word();
+  if (err == nullptr) return ATTN_ERR_CUDA;
+  attn::timeout_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      err, static_cast<unsigned long long>(limit_ms) * 1000000ull);
+  return from_cuda(cudaGetLastError());
 }
 
 attn_status_t attn_device_status(int clear) {

@@ -68,22 +68,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait until the phase of `bar` with parity `parity` has completed.  Gives up
-// after ATTN_WAIT_NS, or at once if *abort is already set; returns false then.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          unsigned int* err) {
+// after limit_ns, or at once if *abort is already set; returns false then,
+// having recorded ATTN_ERRBIT_TIMEOUT and set *abort for the other roles.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                              unsigned int* err, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0u) {
       if (abort != nullptr && *abort) return false;
-      if (globaltimer_ns() - t0 > ATTN_WAIT_NS) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         record_error(err, ATTN_ERRBIT_TIMEOUT);
         if (abort != nullptr) *abort = 1;
         return false;
       }
     }
   }
+}
+
+// mbar_wait_for with the library's limit, ATTN_WAIT_NS.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          unsigned int* err) {
+  return mbar_wait_for(bar, parity, abort, err, ATTN_WAIT_NS);
 }
 
 // ----------------------------------------------------------------- TMA

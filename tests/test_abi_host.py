@@ -217,3 +217,9 @@ def test_fp8_append_argument_validation():
     assert call(vs=float("inf")) == 1
     assert call(kp=None) == 1
     assert call(D=100) == 2
+
+
+def test_selftest_timeout_argument_validation():
+    lib = _lib()
+    assert lib.attn_selftest_wait_timeout(0, None) == 1
+    assert lib.attn_selftest_wait_timeout(1001, None) == 1
