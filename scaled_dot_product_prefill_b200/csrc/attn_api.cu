@@ -65,7 +65,8 @@ attn_status_t check_prefill(const void* q, const void* k, const void* v, const v
   if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
   if (B == 0 || Hq == 0 || Sq == 0) return ATTN_OK;  // nothing to do (checked again by the caller)
   if (Hkv == 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
-  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return ATTN_ERR_INVALID_ARG;
+  // with no keys (Skv == 0) k and v are never read and may be null
+  if (q == nullptr || out == nullptr || (Skv > 0 && (k == nullptr || v == nullptr))) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ATTN_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
   if (window > 0 && !causal) return ATTN_ERR_UNSUPPORTED;

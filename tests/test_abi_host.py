@@ -223,3 +223,13 @@ def test_selftest_timeout_argument_validation():
     lib = _lib()
     assert lib.attn_selftest_wait_timeout(0, None) == 1
     assert lib.attn_selftest_wait_timeout(1001, None) == 1
+
+
+@pytest.mark.parametrize("fn", ["attn_prefill", "attn_prefill_f32"])
+def test_prefill_without_keys_accepts_null_k_and_v(fn):
+    lib = _lib()
+    # Skv == 0: k and v are never read; the call then needs the GPU to write zeros, so on a
+    # machine without one it gets past validation and fails at the CUDA call, not as INVALID_ARG
+    st = prefill(lib, fn, k=None, v=None, Skv=0)
+    assert st in (0, 3)
+    assert prefill(lib, fn, k=None, v=None, Skv=16) == 1
