@@ -1,5 +1,4 @@
 """Edge cases of the entry points on the GPU: calls with no keys at all."""
-import numpy as np
 import pytest
 import torch
 

@@ -1,6 +1,5 @@
 """Failure detection on the GPU without a fault: a bounded wait that nothing completes gives up,
 the host reads the timeout from the device error word, and the context stays usable."""
-import numpy as np
 import pytest
 import torch
 
