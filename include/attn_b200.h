@@ -34,6 +34,8 @@
  *                                     returns the pair (output, lse)).
  *   attn_prefill_paged                chunked prefill whose keys and values sit
  *                                     in the paged cache.
+ *   attn_prefill_host                 the prefill from and to host memory, its
+ *                                     copies overlapped with the kernels.
  *   attn_decode_paged_fp8             the decode over a cache of 8-bit E4M3
  *                                     codes (not on the pages: a storage
  *                                     variant).
@@ -46,8 +48,9 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  * - Pointers named q, k, v, out, k_pool, v_pool, page_table, seq_lens and
- *   workspace are DEVICE pointers of the current CUDA device, 16-byte
- *   aligned, owned by the caller.  The library never allocates or frees
+ *   workspace (and the *_dev buffers) are DEVICE pointers of the current
+ *   CUDA device, 16-byte aligned, owned by the caller; *_host buffers are
+ *   host memory.  The library never allocates or frees
  *   device memory and keeps no state between calls (re-entrant; the one
  *   exception, attn_decode_paged_noalloc, is described at its declaration).
  * - bf16 means IEEE bfloat16 stored in 16 bits; inputs are read as bf16,
@@ -143,6 +146,44 @@ attn_status_t attn_prefill(const void* q, const void* k, const void* v, void* ou
 attn_status_t attn_prefill_lse(const void* q, const void* k, const void* v, void* out, float* lse,
                                int B, int Hq, int Hkv, int Sq, int Skv, int D,
                                float scale, int causal, int window, attn_stream_t stream);
+
+/*
+ * attn_prefill_host -- attn_prefill whose inputs and output live in host
+ * memory: the call copies q, k, v to the device, computes, and copies out
+ * back, cutting the work into `chunks` pieces so that the two copy
+ * directions and the kernels overlap.  A piece is a run of consecutive
+ * (batch, kv head) pairs with their query heads; it is contiguous in every
+ * buffer, so each of its transfers is a single copy, and its kernel is the
+ * attn_prefill of those heads, with the same results bit for bit.
+ *
+ * q_host, k_host, v_host, out_host : host buffers with the layouts of
+ *     attn_prefill.  Page-locked memory (cudaHostAlloc, cudaHostRegister)
+ *     is needed for the copies to overlap anything; pageable memory gives
+ *     the same results, copied synchronously.  The host must not touch
+ *     out_host (nor change the inputs) until `stream` has completed.
+ * q_dev, k_dev, v_dev, out_dev : device buffers of the same sizes, owned by
+ *     the caller (the library allocates nothing), 16-byte aligned; their
+ *     contents are overwritten.  k/v buffers may be null when Skv == 0.
+ * chunks : pieces, 1 .. B * Hkv; 0 = two (one if B * Hkv == 1).  The
+ *     host link bounds the call and each piece adds some copy and launch
+ *     latency, so a few pieces do best.
+ * stream : the stream of the kernels.  When `stream` completes, every copy
+ *     of the call has completed; the copies start only after work that was
+ *     on `stream` before the call.
+ * copy_in, copy_out : streams for the host-to-device and device-to-host
+ *     copies, or NULL to use `stream` (no overlap).  For overlap they must
+ *     be distinct from `stream` and from each other.
+ * B, Hq, Hkv, Sq, Skv, D, scale, causal, window : as attn_prefill.
+ * Errors: as attn_prefill (the device buffers take the place of q, k, v,
+ * out in the checks); ATTN_ERR_INVALID_ARG for a null host buffer or chunks
+ * out of range; ATTN_ERR_CUDA if a copy, event or launch call fails, in
+ * which case the pieces enqueued before the failure stay enqueued.
+ */
+attn_status_t attn_prefill_host(const void* q_host, const void* k_host, const void* v_host, void* out_host,
+                                void* q_dev, void* k_dev, void* v_dev, void* out_dev,
+                                int B, int Hq, int Hkv, int Sq, int Skv, int D,
+                                float scale, int causal, int window, int chunks,
+                                attn_stream_t stream, attn_stream_t copy_in, attn_stream_t copy_out);
 
 /*
  * attn_prefill_f32 -- the same operation with fp32 inputs and output, fp32

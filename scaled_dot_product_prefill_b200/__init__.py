@@ -9,5 +9,5 @@ from .api import (AttnError, PagePool, attn_decode_paged, attn_decode_paged_noal
                   attn_decode_paged_fp8, attn_decode_paged_workspace_size, attn_kv_append,
                   attn_kv_append_fp8,
                   attn_device_status, attn_prefill, attn_prefill_f32, attn_prefill_f32_lse, attn_prefill_lse,
-                  attn_prefill_paged,
+                  attn_prefill_host, attn_prefill_paged,
                   attn_status_string, attn_version)

@@ -22,6 +22,7 @@ PROTOTYPES = {
     "attn_prefill_lse": (_c_int, [_vp] * 5 + [_c_int] * 6 + [_c_float, _c_int, _c_int, _vp]),
     "attn_prefill_f32_lse": (_c_int, [_vp] * 5 + [_c_int] * 6 + [_c_float, _c_int, _c_int, _vp]),
     "attn_prefill_paged": (_c_int, [_vp] * 5 + [_c_int] * 9 + [_c_float, _c_int, _c_int, _vp, _vp, _vp]),
+    "attn_prefill_host": (_c_int, [_vp] * 8 + [_c_int] * 6 + [_c_float, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
     "attn_decode_paged": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 8 + [_c_float, _c_int, _vp, _c_size,
                                                                           _vp, _vp]),
     "attn_decode_paged_fp8": (_c_int, [_vp] * 5 + [_c_int] * 8 + [_c_float] * 3 + [_c_int, _vp, _c_size, _vp, _vp]),

@@ -14,7 +14,7 @@ from . import _lib
 from ._lib import AttnError
 
 __all__ = ["attn_prefill", "attn_prefill_f32", "attn_prefill_lse", "attn_prefill_f32_lse",
-           "attn_prefill_paged", "attn_decode_paged", "attn_decode_paged_noalloc",
+           "attn_prefill_paged", "attn_prefill_host", "attn_decode_paged", "attn_decode_paged_noalloc",
            "attn_decode_paged_workspace_size", "attn_decode_paged_fp8", "attn_kv_append", "attn_kv_append_fp8",
            "PagePool",
            "attn_device_status", "attn_selftest_wait_timeout", "attn_status_string", "attn_version", "AttnError"]
@@ -96,6 +96,72 @@ def _prefill(name, dtype, q, k, v, causal, window, scale, out, stream):
 def attn_prefill(q, k, v, *, causal=False, window=0, scale=None, out=None, stream=None):
     """bf16 prefill: q [B,Hq,Sq,D], k/v [B,Hkv,Skv,D] -> out [B,Hq,Sq,D] (tcgen05 kernel)."""
     return _prefill("attn_prefill", torch.bfloat16, q, k, v, causal, window, scale, out, stream)
+
+
+_COPY_STREAMS: dict = {}
+
+
+def _copy_streams(dev):
+    """The (host-to-device, device-to-host) copy streams of a device, created on first use."""
+    pair = _COPY_STREAMS.get(dev)
+    if pair is None:
+        with torch.cuda.device(dev):
+            pair = (torch.cuda.Stream(), torch.cuda.Stream())
+        _COPY_STREAMS[dev] = pair
+    return pair
+
+
+def attn_prefill_host(q, k, v, *, causal=False, window=0, scale=None, out=None, chunks=0, device_buffers=None,
+                      stream=None, copy_streams="auto"):
+    """bf16 prefill whose q [B,Hq,Sq,D], k/v [B,Hkv,Skv,D] and output are host (CPU) tensors.
+
+    The C call copies the inputs to the device, runs the prefill and copies
+    the output back, in `chunks` pieces (0: two) so that the copies overlap
+    the kernels; page-locked host tensors (``pin_memory()``) are needed for
+    the overlap.  `device_buffers` = (q_dev, k_dev, v_dev, out_dev) CUDA
+    tensors of the same shapes, allocated here if None.  `copy_streams` =
+    (copy_in, copy_out) torch streams, "auto" for two per device, or None to
+    copy on `stream`.  The returned host tensor is complete once `stream`
+    (default: the current stream) has completed.
+    """
+    for t, name in ((q, "q"), (k, "k"), (v, "v")):
+        if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 host tensor")
+    B, Hq, Sq, D = q.shape
+    _, Hkv, Skv, _ = k.shape
+    _expect(k, "k", (B, Hkv, Skv, D), torch.bfloat16)
+    _expect(v, "v", (B, Hkv, Skv, D), torch.bfloat16)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=q.is_pinned())
+    if out.is_cuda or not out.is_contiguous():
+        raise ValueError("out must be a contiguous host tensor")
+    _expect(out, "out", q.shape, torch.bfloat16)
+    dev = torch.cuda.current_device()
+    if device_buffers is None:
+        device_buffers = (torch.empty(q.shape, dtype=torch.bfloat16, device=dev),
+                          torch.empty(k.shape, dtype=torch.bfloat16, device=dev),
+                          torch.empty(v.shape, dtype=torch.bfloat16, device=dev),
+                          torch.empty(q.shape, dtype=torch.bfloat16, device=dev))
+    qd, kd, vd, od = device_buffers
+    for t, ref, name in ((qd, q, "q_dev"), (kd, k, "k_dev"), (vd, v, "v_dev"), (od, q, "out_dev")):
+        _expect(t, name, ref.shape, torch.bfloat16)
+    _need_cuda(qd, kd, vd, od)
+    if copy_streams == "auto":
+        copy_streams = _copy_streams(dev)
+    cin, cout = copy_streams if copy_streams is not None else (None, None)
+    for t in (qd, kd, vd, od):   # the copy streams use the buffers too: keep them from early reuse
+        for cs in (cin, cout):
+            if cs is not None:
+                t.record_stream(cs)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    _check("attn_prefill_host",
+           _lib.load().attn_prefill_host(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(qd), _ptr(kd), _ptr(vd),
+                                         _ptr(od), B, Hq, Hkv, Sq, Skv, D, float(scale), int(bool(causal)),
+                                         int(window), int(chunks), _stream(stream),
+                                         None if cin is None else ctypes_void(cin.cuda_stream),
+                                         None if cout is None else ctypes_void(cout.cuda_stream)))
+    return out
 
 
 def attn_prefill_f32(q, k, v, *, causal=False, window=0, scale=None, out=None, stream=None):

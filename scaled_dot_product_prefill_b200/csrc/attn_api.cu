@@ -92,7 +92,7 @@ const char* attn_status_string(attn_status_t s) {
   return "ATTN_ERR_UNKNOWN";
 }
 
-int attn_version(void) { return 102; }
+int attn_version(void) { return 103; }
 
 }  // extern "C"
 
@@ -178,6 +178,75 @@ attn_status_t attn_prefill_paged(const void* q, const void* k_pool, const void* 
   return from_cuda(attn::launch_prefill_tc_paged(q, k_pool, v_pool, page_table, seq_lens, page_size, B, Hq, Hkv, Sq,
                                                  D, num_pages, max_pages, max_seq_len, scale, causal, window, out, lse,
                                                  attn::device_error_word(), s));
+}
+
+// attn_prefill from and to host memory.  The work is cut into pieces of
+// consecutive (batch, kv head) pairs, each with its query heads: a piece is
+// contiguous in q, k, v and out, so each of its transfers is one copy, and
+// its kernel is an attn_prefill over one batch element of Hkv' = pairs kv
+// heads.  Piece i's input copy (copy_in) overlaps piece i-1's kernel
+// (stream) and piece i-2's output copy (copy_out).
+attn_status_t attn_prefill_host(const void* q_host, const void* k_host, const void* v_host, void* out_host,
+                                void* q_dev, void* k_dev, void* v_dev, void* out_dev, int B, int Hq, int Hkv,
+                                int Sq, int Skv, int D, float scale, int causal, int window, int chunks,
+                                attn_stream_t stream, attn_stream_t copy_in, attn_stream_t copy_out) {
+  attn_status_t st = check_prefill(q_dev, k_dev, v_dev, out_dev, B, Hq, Hkv, Sq, Skv, D, scale, causal, window);
+  if (st != ATTN_OK || B == 0 || Hq == 0 || Sq == 0) return st;
+  if (q_host == nullptr || out_host == nullptr || (Skv > 0 && (k_host == nullptr || v_host == nullptr)))
+    return ATTN_ERR_INVALID_ARG;
+  const long long units = static_cast<long long>(B) * Hkv;   // (batch, kv head) pairs
+  const int G = Hq / Hkv;
+  const size_t q_unit = static_cast<size_t>(G) * Sq * D * 2;   // bytes of q (and out) per pair
+  const size_t kv_unit = static_cast<size_t>(Skv) * D * 2;     // bytes of k (and v) per pair
+  if (chunks < 0 || chunks > units) return ATTN_ERR_INVALID_ARG;
+  // The host link bounds this call, not the kernels, and every piece adds some
+  // tens of microseconds of copy and launch latency: two pieces (the second
+  // one's input copy overlapping the first one's kernel and output copy) is
+  // the default.
+  if (chunks == 0) chunks = units >= 2 ? 2 : 1;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaStream_t si = copy_in != nullptr ? reinterpret_cast<cudaStream_t>(copy_in) : s;
+  cudaStream_t so = copy_out != nullptr ? reinterpret_cast<cudaStream_t>(copy_out) : s;
+  cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};   // entry / inputs of a piece on the device / its output ready
+  for (auto& e : ev)
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) st = ATTN_ERR_CUDA;
+  // the copies wait for earlier work on `stream` (which may still use the device buffers)
+  if (st == ATTN_OK && (cudaEventRecord(ev[0], s) != cudaSuccess || cudaStreamWaitEvent(si, ev[0], 0) != cudaSuccess ||
+                        cudaStreamWaitEvent(so, ev[0], 0) != cudaSuccess))
+    st = ATTN_ERR_CUDA;
+  const char* qh = static_cast<const char*>(q_host);
+  const char* kh = static_cast<const char*>(k_host);
+  const char* vh = static_cast<const char*>(v_host);
+  char* oh = static_cast<char*>(out_host);
+  char* qd = static_cast<char*>(q_dev);
+  char* kd = static_cast<char*>(k_dev);
+  char* vd = static_cast<char*>(v_dev);
+  char* od = static_cast<char*>(out_dev);
+  for (int c = 0; c < chunks && st == ATTN_OK; ++c) {
+    const long long u0 = units * c / chunks, u1 = units * (c + 1) / chunks;
+    if (u1 <= u0) continue;
+    const size_t n = static_cast<size_t>(u1 - u0);
+    const size_t qo = static_cast<size_t>(u0) * q_unit, ko = static_cast<size_t>(u0) * kv_unit;
+    if (cudaMemcpyAsync(qd + qo, qh + qo, n * q_unit, cudaMemcpyHostToDevice, si) != cudaSuccess ||
+        (kv_unit > 0 && (cudaMemcpyAsync(kd + ko, kh + ko, n * kv_unit, cudaMemcpyHostToDevice, si) != cudaSuccess ||
+                         cudaMemcpyAsync(vd + ko, vh + ko, n * kv_unit, cudaMemcpyHostToDevice, si) != cudaSuccess)) ||
+        cudaEventRecord(ev[1], si) != cudaSuccess || cudaStreamWaitEvent(s, ev[1], 0) != cudaSuccess) {
+      st = ATTN_ERR_CUDA;
+      break;
+    }
+    st = prefill_bf16(qd + qo, kv_unit > 0 ? kd + ko : nullptr, kv_unit > 0 ? vd + ko : nullptr, od + qo, nullptr, 1,
+                      static_cast<int>(n) * G, static_cast<int>(n), Sq, Skv, D, scale, causal, window, stream);
+    if (st != ATTN_OK) break;
+    if (cudaEventRecord(ev[2], s) != cudaSuccess || cudaStreamWaitEvent(so, ev[2], 0) != cudaSuccess ||
+        cudaMemcpyAsync(oh + qo, od + qo, n * q_unit, cudaMemcpyDeviceToHost, so) != cudaSuccess)
+      st = ATTN_ERR_CUDA;
+  }
+  // later work on `stream` comes after every copy of this call
+  if (st == ATTN_OK && (cudaEventRecord(ev[2], so) != cudaSuccess || cudaStreamWaitEvent(s, ev[2], 0) != cudaSuccess))
+    st = ATTN_ERR_CUDA;
+  for (auto& e : ev)
+    if (e != nullptr) cudaEventDestroy(e);   // released once the recorded work completes
+  return st;
 }
 
 attn_status_t attn_prefill_f32(const float* q, const float* k, const float* v, float* out, int B, int Hq, int Hkv,

@@ -233,3 +233,21 @@ def test_prefill_without_keys_accepts_null_k_and_v(fn):
     st = prefill(lib, fn, k=None, v=None, Skv=0)
     assert st in (0, 3)
     assert prefill(lib, fn, k=None, v=None, Skv=16) == 1
+
+
+def test_host_prefill_argument_validation():
+    lib = _lib()
+
+    def call(qh=FAKE, kh=FAKE, vh=FAKE, oh=FAKE, qd=FAKE, kd=FAKE, vd=FAKE, od=FAKE, B=2, Hq=4, Hkv=2, D=64,
+             chunks=0, Skv=64):
+        return lib.attn_prefill_host(qh, kh, vh, oh, qd, kd, vd, od, B, Hq, Hkv, 64, Skv, D, 0.125, 1, 0, chunks,
+                                     None, None, None)
+
+    assert call(qh=None) == 1                    # host buffers are required
+    assert call(oh=None) == 1
+    assert call(od=None) == 1                    # and the device ones
+    assert call(qd=MISALIGNED) == 1
+    assert call(chunks=-1) == 1
+    assert call(chunks=5) == 1                   # more pieces than (batch, kv head) pairs (2 x 2)
+    assert call(D=96) == 2
+    assert call(B=0, qh=None, oh=None, qd=None, od=None) == 0   # empty problem
