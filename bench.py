@@ -199,6 +199,23 @@ def job_rate(units_per_rank, world, ms):
     return world * float(units_per_rank) / (ms * 1e-3)
 
 
+def arm_config(world, seq_lens):
+    """The workload description both arms print (decode sequence lengths of rank 0's seed)."""
+    spec, dspec = PREFILL, DECODE
+    return {
+        "workload": f"{spec.name} + {dspec.name}",
+        "prefill": {"B": spec.B, "Hq": spec.Hq, "Hkv": spec.Hkv, "S": spec.Sq, "D": spec.D,
+                    "causal": spec.causal, "window": spec.window, "flops": workloads.prefill_flops(spec)},
+        "decode": {"N": dspec.N, "Hq": dspec.Hq, "Hkv": dspec.Hkv, "D": dspec.D,
+                   "page_size": dspec.page_size, "len_range": list(dspec.len_range),
+                   "sum_len": int(np.sum(seq_lens)),
+                   "kv_bytes": workloads.kv_bytes(seq_lens, dspec.Hkv, dspec.D),
+                   "bytes": workloads.decode_bytes(seq_lens, dspec.Hq, dspec.Hkv, dspec.D, dspec.page_size)},
+        "l2": "prefill: 256 MiB write before each call; decode: 1.1 GB K/V > 126 MB L2",
+        "parallelism": f"replicas x{world}",
+    }
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
 
@@ -229,7 +246,6 @@ def run_ours(args, rank, world, local_rank):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     p_flops = workloads.prefill_flops(spec)
     d_bytes = workloads.decode_bytes(pd.seq_lens.numpy(), dspec.Hq, dspec.Hkv, dspec.D, dspec.page_size)
-    d_kv_bytes = workloads.kv_bytes(pd.seq_lens.numpy(), dspec.Hkv, dspec.D)
 
     def step(ev=None):
         flush.zero_()
@@ -323,16 +339,7 @@ def run_ours(args, rank, world, local_rank):
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic (seeded N(0,1), bf16)",
-            "config": {
-                "workload": f"{spec.name} + {dspec.name}",
-                "prefill": {"B": spec.B, "Hq": spec.Hq, "Hkv": spec.Hkv, "S": spec.Sq, "D": spec.D,
-                            "causal": spec.causal, "window": spec.window, "flops": p_flops},
-                "decode": {"N": dspec.N, "Hq": dspec.Hq, "Hkv": dspec.Hkv, "D": dspec.D,
-                           "page_size": dspec.page_size, "len_range": list(dspec.len_range),
-                           "sum_len": int(pd.seq_lens.sum()), "kv_bytes": d_kv_bytes, "bytes": d_bytes},
-                "l2": "prefill: 256 MiB write before each call; decode: 1.1 GB K/V > 126 MB L2",
-                "parallelism": f"replicas x{world}",
-            },
+            "config": arm_config(world, pd.seq_lens.numpy()),
             "roofline": {"bound": "tensor", "achieved": round(ach_t, 2), "peak": peak_t, "unit": "TFLOP/s",
                          "frac": round(ach_t / peak_t, 4), "traffic": traffic,
                          "kernel": "prefill_tc_kernel<64, false, 0>", "peak_kind": f"bf16 burst, {peak_kind}"},
@@ -561,7 +568,7 @@ def reference_line(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1), bf16 values upcast)",
-        "config": {"workload": f"{PREFILL.name} (oracle sample)", "parallelism": "host cores"},
+        "config": arm_config(world, inputs.draw_seq_lens(DECODE.N, DECODE.seed, DECODE.len_range).numpy()),
         "cpu_baseline": {"value": round(v, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

@@ -81,6 +81,12 @@ class PagedInputs:
         return int(self.seq_lens.max().item()) if self.seq_lens.numel() else 0
 
 
+def draw_seq_lens(N: int, seed: int, len_range=(512, 8192)) -> torch.Tensor:
+    """The sequence lengths ``paged_inputs`` draws for ``seed``: integers uniform in ``len_range`` (inclusive)."""
+    lo, hi = len_range
+    return torch.randint(int(lo), int(hi) + 1, (N,), generator=_gen(int(seed) * 16 + 3), dtype=torch.int64)
+
+
 def paged_inputs(N, Hq, Hkv, D, page_size: int, seed: int, *, seq_lens=None,
                  len_range=(512, 8192), spare_pages: int = 0, poison: bool = False,
                  max_pages: int | None = None, dtype: str = "bf16") -> PagedInputs:
@@ -95,9 +101,7 @@ def paged_inputs(N, Hq, Hkv, D, page_size: int, seed: int, *, seq_lens=None,
     """
     base = int(seed) * 16
     if seq_lens is None:
-        lo, hi = len_range
-        seq_lens = torch.randint(int(lo), int(hi) + 1, (N,), generator=_gen(base + 3),
-                                 dtype=torch.int64)
+        seq_lens = draw_seq_lens(N, seed, len_range)
     seq_lens = torch.as_tensor(seq_lens, dtype=torch.int64).reshape(-1)
     assert seq_lens.numel() == N
     n_pages_seq = [(int(L) + page_size - 1) // page_size for L in seq_lens.tolist()]
