@@ -77,3 +77,19 @@ def test_single_process_keeps_its_own_times_and_rates_count_every_rank():
 def test_gloo_is_available():
     assert dist.is_available() and dist.is_gloo_available()
     assert torch.multiprocessing.get_all_start_methods()
+
+
+def test_both_arms_describe_the_same_workload():
+    """The reference arm draws the decode lengths without building the pools; they must be the lengths the
+    timed arm's generated cache has."""
+    import numpy as np
+
+    from scaled_dot_product_prefill_b200 import inputs
+
+    for seed, rng in ((5, (512, 8192)), (1234, (1, 40))):
+        p = inputs.paged_inputs(6, 8, 2, 64, 16, seed=seed, len_range=rng)
+        assert np.array_equal(p.seq_lens.numpy(), inputs.draw_seq_lens(6, seed, rng).numpy())
+    d = bench.DECODE
+    lens = inputs.draw_seq_lens(d.N, d.seed, d.len_range).numpy()
+    cfg = bench.arm_config(1, lens)
+    assert cfg["decode"]["sum_len"] == int(lens.sum()) and cfg["workload"].startswith(bench.PREFILL.name)
