@@ -316,6 +316,7 @@ def run_ours(args, rank, world, local_rank):
         extra = other_workloads(dev, peaks)
         extra.update(append_workloads(dev, peaks))
         extra.update(fp8_decode_workload(dev, peaks))
+        extra.update(paged_prefill_workload(dev, peaks))
 
     result = None
     if rank == 0:
@@ -505,11 +506,34 @@ def other_workloads(dev, peaks):
     return res
 
 
+def paged_prefill_workload(dev, peaks):
+    """The chunked prefill over a paged cache (bottom-right causal), one timing."""
+    import torch
+
+    from scaled_dot_product_prefill_b200 import api
+
+    spec = workloads.EXTRA_WORKLOADS["chunked_prefill_paged_gqa"]
+    p = inputs.paged_inputs(spec.B, spec.Hq, spec.Hkv, spec.D, spec.page_size, spec.seed, seq_lens=[spec.L] * spec.B)
+    q = inputs.normal((spec.B, spec.Hq, spec.Sq, spec.D), seed=spec.seed + 1).to(dev)
+    kp, vp, pt, sl = (t.to(dev) for t in (p.k_pool, p.v_pool, p.page_table, p.seq_lens))
+    out = torch.empty_like(q)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    ms = time_call(lambda: api.attn_prefill_paged(q, kp, vp, pt, sl, max_seq_len=spec.L, causal=True,
+                                                  scale=spec.scale, out=out), 20, flush)
+    ach = workloads.paged_prefill_flops(spec) / (ms * 1e-3) / 1e12
+    res = {spec.name: {"ms": round(ms, 5), "TFLOP/s": round(ach, 2),
+                       "frac_of_bf16_peak": round(ach / float(peaks["bf16_tflops"]), 4),
+                       "l2": "256 MB write before each call"}}
+    del q, kp, vp, pt, sl, out, flush
+    torch.cuda.empty_cache()
+    return res
+
+
 def profile_case(name, calls):
     """Run one workload ``calls`` times and nothing else, for a profiler capture of its kernels.
 
-    ``name`` is a prefill workload of ``workloads.WORKLOADS``, ``paged_decode_gqa``, or
-    ``paged_decode_gqa_fp8`` (the same decode over an 8-bit cache).  Prints one line with the
+    ``name`` is a prefill workload of ``workloads.WORKLOADS``, ``paged_decode_gqa``,
+    ``paged_decode_gqa_fp8`` (the same decode over an 8-bit cache), or ``chunked_prefill_paged_gqa``.  Prints one line with the
     mean CUDA-event time, which is not a benchmark number when taken under a profiler.
     """
     import torch
@@ -537,6 +561,15 @@ def profile_case(name, calls):
         else:
             fn = lambda: api.attn_decode_paged(dq, kp, vp, pt, sl, max_seq_len=pd.max_seq_len, scale=spec.scale,
                                                workspace=ws, out=out)
+    elif name in workloads.EXTRA_WORKLOADS:
+        spec = workloads.EXTRA_WORKLOADS[name]
+        pp = inputs.paged_inputs(spec.B, spec.Hq, spec.Hkv, spec.D, spec.page_size, spec.seed,
+                                 seq_lens=[spec.L] * spec.B)
+        q = inputs.normal((spec.B, spec.Hq, spec.Sq, spec.D), seed=spec.seed + 1).to(dev)
+        kp, vp, pt, sl = (t.to(dev) for t in (pp.k_pool, pp.v_pool, pp.page_table, pp.seq_lens))
+        out = torch.empty_like(q)
+        fn = lambda: api.attn_prefill_paged(q, kp, vp, pt, sl, max_seq_len=spec.L, causal=True, scale=spec.scale,
+                                            out=out)
     else:
         spec = workloads.WORKLOADS[name]
         pi = inputs.prefill_inputs(spec.B, spec.Hq, spec.Hkv, spec.Sq, spec.Skv, spec.D, spec.seed, spec.dtype)

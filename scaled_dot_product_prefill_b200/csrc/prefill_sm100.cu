@@ -285,10 +285,20 @@ __global__ void __launch_bounds__(Cfg<D, V>::THREADS, Cfg<D, V>::MINB)
    if constexpr (C::SPLIT_REGS) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::PRODUCER_REGS));
    if (warp == kTmaWarp) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      prefetch_tmap(&tmap_q);
-      prefetch_tmap(&tmap_k);
-      prefetch_tmap(&tmap_v);
+    // Dense: one thread.  Paged: the whole warp, so that the page-table
+    // entries of a tile are read by one load and its page boxes issued by
+    // one instruction (lane 0 still arms the barriers and loads Q).
+    if (PAGED || lane == 0) {
+      const bool lead = (lane == 0);
+      auto uni = [&](bool v) -> bool {   // one outcome for the whole warp
+        if constexpr (PAGED) return __all_sync(0xffffffffu, v);
+        return v;
+      };
+      if (lead) {
+        prefetch_tmap(&tmap_q);
+        prefetch_tmap(&tmap_k);
+        prefetch_tmap(&tmap_v);
+      }
       int n = 0, qn = 0;
       bool ok = true;
       for (int r = 0; r < n_rounds && ok; ++r) {
@@ -297,18 +307,20 @@ __global__ void __launch_bounds__(Cfg<D, V>::THREADS, Cfg<D, V>::MINB)
         const Item it = make_item<BN, PAGED>(p, k);
         if (it.hi_all <= it.lo_all) continue;
         const int qb = qn % QBUF;
-        if (qn >= QBUF && !(ok = mbar_wait(&q_empty[qb], ((qn / QBUF) - 1) & 1, abort_flag, p.err))) break;
-        mbar_arrive_expect_tx(&q_full[qb], NQ * C::Q_BYTES);
-        for (int i = 0; i < NQ; ++i)
-          for (int a = 0; a < C::KATOMS; ++a)
-            tma_load_3d(sQ + ((qb * NQ + i) * C::KATOMS + a) * BM * 128, &tmap_q, &q_full[qb], a * 64,
-                        it.q_row0 + BM * i, it.bh);
+        if (qn >= QBUF && !(ok = uni(mbar_wait(&q_empty[qb], ((qn / QBUF) - 1) & 1, abort_flag, p.err)))) break;
+        if (lead) {
+          mbar_arrive_expect_tx(&q_full[qb], NQ * C::Q_BYTES);
+          for (int i = 0; i < NQ; ++i)
+            for (int a = 0; a < C::KATOMS; ++a)
+              tma_load_3d(sQ + ((qb * NQ + i) * C::KATOMS + a) * BM * 128, &tmap_q, &q_full[qb], a * 64,
+                          it.q_row0 + BM * i, it.bh);
+        }
         ++qn;
         const int kv_plane = it.b * p.Hkv + it.g;
         auto load = [&](bool is_v, int j) -> bool {   // next ring slot <- K_j or V_j
           const int st = n % STAGES;
-          if (!mbar_wait(&empty[st], ((n / STAGES) & 1) ^ 1, abort_flag, p.err)) return false;
-          mbar_arrive_expect_tx(&full[st], C::TILE_BYTES);
+          if (!uni(mbar_wait(&empty[st], ((n / STAGES) & 1) ^ 1, abort_flag, p.err))) return false;
+          if (lead) mbar_arrive_expect_tx(&full[st], C::TILE_BYTES);
           const CUtensorMap* tm = is_v ? &tmap_v : &tmap_k;
           if constexpr (!PAGED) {
             for (int a = 0; a < C::KATOMS; ++a)
@@ -318,30 +330,23 @@ __global__ void __launch_bounds__(Cfg<D, V>::THREADS, Cfg<D, V>::MINB)
             // box lands at its row offset inside the swizzled tile, so the MMA
             // sees the same layout as a dense load
             // boxes that start past the sequence end read no page: their plane
-            // coordinate is past the pool, so the copy fills them with zeros
+            // coordinate is past the pool, so the copy fills them with zeros.
+            // Lane rb + nb * a copies box rb of swizzle atom a (at most 8 x 2).
+            __syncwarp();   // the barrier is armed before any box can land
             const int nb = BN / p.box_rows;
-            int phys[8];
-#pragma unroll
-            for (int rb = 0; rb < 8; ++rb) {
-              if (rb >= nb) break;
+            if (lane < nb * C::KATOMS) {
+              const int rb = lane % nb, a = lane / nb;
               const int key0 = j * BN + rb * p.box_rows;
-              const int pg = key0 / p.page_size;
-              phys[rb] = (key0 < it.skv) ? p.page_table[static_cast<size_t>(it.b) * p.max_pages + pg] : 0;
-            }
-#pragma unroll
-            for (int rb = 0; rb < 8; ++rb) {
-              if (rb >= nb) break;
-              const int key0 = j * BN + rb * p.box_rows;
-              int ph = phys[rb];
-              if (key0 >= it.skv) {
-                ph = p.num_pages;                   // plane ph * Hkv + g is past the pool's planes
-              } else if (ph < 0 || ph >= p.num_pages) {   // never read outside the pool
-                record_error(p.err, ATTN_ERRBIT_BADPAGE);
-                ph = 0;
+              int ph = p.num_pages;                 // plane ph * Hkv + g is past the pool's planes
+              if (key0 < it.skv) {
+                ph = p.page_table[static_cast<size_t>(it.b) * p.max_pages + key0 / p.page_size];
+                if (ph < 0 || ph >= p.num_pages) {  // never read outside the pool
+                  record_error(p.err, ATTN_ERRBIT_BADPAGE);
+                  ph = 0;
+                }
               }
-              for (int a = 0; a < C::KATOMS; ++a)
-                tma_load_3d(sRing + st * C::TILE_BYTES + a * BN * 128 + rb * p.box_rows * 128, tm, &full[st],
-                            a * 64, key0 % p.page_size, ph * p.Hkv + it.g);
+              tma_load_3d(sRing + st * C::TILE_BYTES + a * BN * 128 + rb * p.box_rows * 128, tm, &full[st],
+                          a * 64, key0 % p.page_size, ph * p.Hkv + it.g);
             }
           }
           ++n;

@@ -60,6 +60,25 @@ class DecodeSpec:
         return 1.0 / float(np.sqrt(self.D))
 
 
+@dataclass(frozen=True)
+class PagedPrefillSpec:
+    """Chunked prefill over a paged cache: B sequences of L cached tokens each, the last Sq of them new."""
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    L: int
+    Sq: int
+    D: int
+    page_size: int
+    seed: int
+    desc: str = ""
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / float(np.sqrt(self.D))
+
+
 WORKLOADS = {
     "single_head_f32": PrefillSpec(
         "single_head_f32", 1, 1, 1, 256, 256, 64, False, 0, "f32", 1000,
@@ -120,3 +139,17 @@ def decode_bytes(seq_lens, Hq: int, Hkv: int, D: int, page_size: int, elem_bytes
     Lw = np.minimum(L, window) if window and window > 0 else L
     pages = int(((Lw + page_size - 1) // page_size).sum())
     return kv_bytes(L, Hkv, D, elem_bytes, window) + 2 * n * Hq * D * elem_bytes + 4 * pages
+
+
+# Measurement cases beyond the five above (their rows of the scope table are built on top of them).
+EXTRA_WORKLOADS = {
+    "chunked_prefill_paged_gqa": PagedPrefillSpec(
+        "chunked_prefill_paged_gqa", 4, 32, 8, 4096, 1024, 128, 16, 1005,
+        "chunked prefill over a paged cache: 4 sequences of 4096 cached tokens, the last 1024 new, "
+        "Hq=32 Hkv=8 D=128, page 16, pages scattered over the pool, bf16"),
+}
+
+
+def paged_prefill_flops(spec: PagedPrefillSpec) -> int:
+    """The Sq new rows attend causally (bottom-right) over the L cached keys."""
+    return attention_flops(spec.B, spec.Hq, spec.Sq, spec.L, spec.D, True)

@@ -118,3 +118,26 @@ def test_paged_prefill_chunk_at_the_end_of_a_long_cache():
     assert api.attn_device_status(clear=True) == 0
     ref, _ = oracle_paged_prefill(q, p, 1 / np.sqrt(128), True, 0)
     assert_parity(out, ref, "bf16", "20k cache, 512-token chunk")
+
+
+def test_chunked_prefill_workload_on_sampled_rows():
+    """The benchmark's chunked prefill, in the launch it times, checked on sampled rows of four heads."""
+    from scaled_dot_product_prefill_b200 import workloads
+
+    spec = workloads.EXTRA_WORKLOADS["chunked_prefill_paged_gqa"]
+    p = inputs.paged_inputs(spec.B, spec.Hq, spec.Hkv, spec.D, spec.page_size, spec.seed, seq_lens=[spec.L] * spec.B)
+    q = inputs.normal((spec.B, spec.Hq, spec.Sq, spec.D), seed=spec.seed + 1)
+    dev = [t.cuda() for t in (p.k_pool, p.v_pool, p.page_table, p.seq_lens)]
+    out = api.attn_prefill_paged(q.cuda(), *dev, max_seq_len=spec.L, causal=True, scale=spec.scale)
+    torch.cuda.synchronize()
+    assert api.attn_device_status(clear=True) == 0
+    out = out.cpu()
+    rng = np.random.default_rng(spec.seed)
+    G = spec.Hq // spec.Hkv
+    for b, h in [(0, 0), (spec.B - 1, spec.Hq - 1), (1, G), (2, spec.Hq // 2 + 1)]:
+        rows = sorted(set([0, 1, 127, 128, spec.Sq - 1]) | set(rng.integers(0, spec.Sq, 40).tolist()))
+        g = h // G
+        K = sdpa.gather_pages(p.k_pool, p.page_table[b].numpy(), spec.L, spec.page_size)[:, g]
+        V = sdpa.gather_pages(p.v_pool, p.page_table[b].numpy(), spec.L, spec.page_size)[:, g]
+        ref = sdpa.attention_rows(q[b, h, rows], K, V, rows, spec.Sq, spec.scale, True)
+        assert_parity(out[b, h, rows], ref, "bf16", f"{spec.name} b={b} h={h}")

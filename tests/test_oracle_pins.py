@@ -310,6 +310,11 @@ def test_visible_pair_counts_match_the_oracle_predicate():
     # the sliding-window workload: min(i + 1, 4096) keys per query over 16384 queries
     assert workloads.visible_pairs(16384, 16384, True, 4096) == 58_722_304
     assert workloads.prefill_flops(workloads.WORKLOADS["gqa_swa_16k"]) == 4 * 128 * 32 * 58_722_304
+    # the chunked prefill: query i of the last 1024 of 4096 tokens sees 3072 + i + 1 keys
+    spec = workloads.EXTRA_WORKLOADS["chunked_prefill_paged_gqa"]
+    pairs = 1024 * 3072 + 1024 * 1025 // 2
+    assert workloads.visible_pairs(1024, 4096, True, 0) == pairs
+    assert workloads.paged_prefill_flops(spec) == 4 * 128 * 4 * 32 * pairs
 
 
 def test_lse_matches_python_log_sum_exp_and_merges_disjoint_key_sets():
