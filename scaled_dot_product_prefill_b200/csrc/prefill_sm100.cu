@@ -16,7 +16,8 @@
 //   warps 0-3  softmax group 0: thread t owns row t of query tile 0
 //   warps 4-7  softmax group 1: the same for query tile 1
 //   warp 8     TMA producer: Q of each item, then K_j / V_j tiles into a ring
-//              of shared-memory slots (128-byte swizzle, no multicast)
+//              of shared-memory slots (128-byte swizzle, no multicast); one
+//              thread for dense K/V, the whole warp for page boxes
 //   warp 9     MMA issuer (one thread) and tensor-memory owner
 //   warps 10-11 idle (complete the third warpgroup for the register split)
 // Tensor memory (512 columns x 128 lanes, fp32):
