@@ -241,9 +241,13 @@ attn_status_t attn_prefill_host(const void* q_host, const void* k_host, const vo
         cudaMemcpyAsync(oh + qo, od + qo, n * q_unit, cudaMemcpyDeviceToHost, so) != cudaSuccess)
       st = ATTN_ERR_CUDA;
   }
-  // later work on `stream` comes after every copy of this call
-  if (st == ATTN_OK && (cudaEventRecord(ev[2], so) != cudaSuccess || cudaStreamWaitEvent(s, ev[2], 0) != cudaSuccess))
-    st = ATTN_ERR_CUDA;
+  // later work on `stream` comes after every copy this call enqueued, also
+  // when a piece failed part way
+  if (ev[1] != nullptr && ev[2] != nullptr) {
+    const bool joined = cudaEventRecord(ev[1], si) == cudaSuccess && cudaStreamWaitEvent(s, ev[1], 0) == cudaSuccess &&
+                        cudaEventRecord(ev[2], so) == cudaSuccess && cudaStreamWaitEvent(s, ev[2], 0) == cudaSuccess;
+    if (!joined && st == ATTN_OK) st = ATTN_ERR_CUDA;
+  }
   for (auto& e : ev)
     if (e != nullptr) cudaEventDestroy(e);   // released once the recorded work completes
   return st;
