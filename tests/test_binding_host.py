@@ -60,3 +60,15 @@ def test_paged_prefill_and_append_refuse_mismatched_tables():
         api.attn_kv_append_fp8(t(2, 2, 5, 64), t(2, 2, 5, 64), kp.view(torch.uint8)[..., :64].contiguous(),
                                kp.view(torch.uint8)[..., :64].contiguous(), t(3, 4, dtype=torch.int32),
                                t(2, dtype=torch.int32), k_scale=1, v_scale=1)
+
+
+def test_host_prefill_refuses_bad_host_tensors_before_touching_the_gpu():
+    q, k, v = t(2, 4, 64, 64), t(2, 2, 64, 64), t(2, 2, 64, 64)
+    with pytest.raises(ValueError, match="q must be"):
+        api.attn_prefill_host(q.float(), k, v)
+    with pytest.raises(ValueError, match="k must be"):
+        api.attn_prefill_host(q, t(2, 2, 64, 128)[..., ::2], v)      # not contiguous
+    with pytest.raises(ValueError, match="v must have shape"):
+        api.attn_prefill_host(q, k, t(2, 2, 65, 64))
+    with pytest.raises(ValueError, match="out must have shape"):
+        api.attn_prefill_host(q, k, v, out=t(2, 4, 64, 32))
