@@ -177,7 +177,8 @@ attn_status_t attn_prefill_lse(const void* q, const void* k, const void* v, void
  * Errors: as attn_prefill (the device buffers take the place of q, k, v,
  * out in the checks); ATTN_ERR_INVALID_ARG for a null host buffer or chunks
  * out of range; ATTN_ERR_CUDA if a copy, event or launch call fails, in
- * which case the pieces enqueued before the failure stay enqueued.
+ * which case the pieces enqueued before the failure stay enqueued and
+ * `stream` still waits for their copies.
  */
 attn_status_t attn_prefill_host(const void* q_host, const void* k_host, const void* v_host, void* out_host,
                                 void* q_dev, void* k_dev, void* v_dev, void* out_dev,
