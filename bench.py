@@ -1,15 +1,18 @@
 """Benchmark of the attention hot path on B200: prefill TFLOP/s and paged-decode KV GB/s.
 
 One step = one pass of the whole path over one batch of synthetic input:
-  1. attn_prefill on the causal MHA GPT-2-small shape (B=8, H=12, S=1024,
-     D=64, bf16; L2 flushed by a 256 MiB write before it), and
+  1. attn_prefill on the causal sliding-window GQA prefill, the largest
+     prefill workload (B=1, Hq=32, Hkv=8, S=16384, W=4096, D=128, bf16;
+     962 GFLOP; 335 MB of q, k, v and out, and a 256 MiB write before it
+     flushes L2), and
   2. attn_decode_paged on the paged GQA decode batch (64 sequences, Hq=32,
      Hkv=8, D=128, L ~ U[512, 8192], 16-token pages; 1.1 GB of K/V, larger
      than L2).
 `value` is the prefill throughput in TFLOP/s (4*D flops per visible
 (query, key) pair); the decode throughput (algorithmic K/V bytes per
 second) is reported beside it with its own roofline.  Each kernel is timed
-with CUDA events on the stream it is launched on.
+with CUDA events on the stream it is launched on.  The other prefill
+workloads are timed after the steps, each with its own roofline entry.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 Under torchrun each rank runs the same per-GPU workload (weak scaling, no
@@ -33,7 +36,7 @@ sys.path.insert(0, ROOT)
 
 from scaled_dot_product_prefill_b200 import inputs, workloads  # noqa: E402
 
-PREFILL = workloads.WORKLOADS["mha_causal_gpt2s"]
+PREFILL = workloads.WORKLOADS["gqa_swa_16k"]
 DECODE = workloads.WORKLOADS["paged_decode_gqa"]
 METRIC = "prefill TFLOP/s & paged-decode KV GB/s on 1 B200, % of roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -141,22 +144,37 @@ def cpu_threads():
         return os.cpu_count() or 1
 
 
+ORACLE_ROWS = 256   # query rows per oracle call in the CPU sample
+
+
 def oracle_prefill_sample(budget_s=8.0):
-    """Float64 oracle on whole (batch, head) slices of the prefill workload until the budget is spent."""
+    """Float64 oracle on blocks of query rows of the prefill workload until the budget is spent.
+
+    Each call is the oracle's attention_rows for ORACLE_ROWS consecutive rows of
+    one head against all of that head's keys, as the oracle computes them;
+    the blocks walk the rows of head 0 from the end (the rows with the most
+    visible keys first).  Work is counted as in the GPU leg: 4*D flops per
+    visible (query, key) pair of the rows done.
+    """
     from oracle import sdpa
 
     spec = PREFILL
-    inp = inputs.prefill_inputs(1, 4, 4, spec.Sq, spec.Skv, spec.D, spec.seed)
+    inp = inputs.prefill_inputs(1, 1, 1, spec.Sq, spec.Skv, spec.D, spec.seed)
+    q, k, v = inp.q[0, 0], inp.k[0, 0], inp.v[0, 0]
+    per_row = workloads.visible_per_row(spec.Sq, spec.Skv, spec.causal, spec.window)
     flops = done = 0
+    n_blocks = (spec.Sq + ORACLE_ROWS - 1) // ORACLE_ROWS
     t0 = time.perf_counter()
     while time.perf_counter() - t0 < budget_s or done == 0:
-        h = done % 4
-        sdpa.attention(inp.q[:, h:h + 1], inp.k[:, h:h + 1], inp.v[:, h:h + 1], spec.scale, spec.causal,
-                       spec.window)
-        flops += workloads.attention_flops(1, 1, spec.Sq, spec.Skv, spec.D, spec.causal, spec.window)
+        blk = n_blocks - 1 - done % n_blocks
+        rows = list(range(blk * ORACLE_ROWS, min(spec.Sq, (blk + 1) * ORACLE_ROWS)))
+        sdpa.attention_rows(q[rows], k, v, rows, spec.Sq, spec.scale, spec.causal, spec.window)
+        flops += 4 * spec.D * int(per_row[rows].sum())
         done += 1
     dt = time.perf_counter() - t0
-    return flops / dt / 1e12, f"{done} (batch, head) slices of {spec.name} ({spec.Sq}x{spec.Skv}, D={spec.D})", dt
+    return (flops / dt / 1e12,
+            f"{done} blocks of {ORACLE_ROWS} query rows of one head of {spec.name} ({spec.Sq}x{spec.Skv}, "
+            f"D={spec.D}, W={spec.window}), each against all {spec.Skv} keys as the oracle evaluates them", dt)
 
 
 def oracle_decode_sample(budget_s=6.0):
@@ -211,7 +229,8 @@ def arm_config(world, seq_lens):
                    "sum_len": int(np.sum(seq_lens)),
                    "kv_bytes": workloads.kv_bytes(seq_lens, dspec.Hkv, dspec.D),
                    "bytes": workloads.decode_bytes(seq_lens, dspec.Hq, dspec.Hkv, dspec.D, dspec.page_size)},
-        "l2": "prefill: 256 MiB write before each call; decode: 1.1 GB K/V > 126 MB L2",
+        "l2": "prefill: 256 MiB write before each call (and 335 MB of q/k/v/out > 126 MB L2); "
+              "decode: 1.1 GB K/V > 126 MB L2",
         "parallelism": f"replicas x{world}",
     }
 
@@ -343,9 +362,11 @@ def run_ours(args, rank, world, local_rank):
             "config": arm_config(world, pd.seq_lens.numpy()),
             "roofline": {"bound": "tensor", "achieved": round(ach_t, 2), "peak": peak_t, "unit": "TFLOP/s",
                          "frac": round(ach_t / peak_t, 4), "traffic": traffic,
-                         "kernel": "prefill_tc_kernel<64, false, 0>", "peak_kind": f"bf16 burst, {peak_kind}"},
+                         "algorithmic_flops": p_flops, "ms": round(pre_ms, 5),
+                         "kernel": f"prefill_tc_kernel<{spec.D}, false>", "peak_kind": f"bf16 burst, {peak_kind}"},
             "roofline_decode": {"bound": "hbm", "achieved": round(ach_d, 1), "peak": peak_h, "unit": "GB/s",
-                                "frac": round(ach_d / peak_h, 4), "traffic": traffic_d,
+                                "frac": round(ach_d / peak_h, 4), "traffic": traffic_d, "algorithmic_bytes": d_bytes,
+                                "ms": round(dec_ms, 5),
                                 "kernel": "decode_split_kernel<128,4,false> + decode_combine_kernel<128>",
                                 "peak_kind": f"HBM copy, {peak_kind}"},
             "decode": {"value": round(job_rate(d_bytes, world, dec_ms) / 1e9, 1), "unit": "GB/s",
@@ -480,6 +501,11 @@ def append_workloads(dev, peaks):
 
 
 def other_workloads(dev, peaks):
+    """The other prefill workloads, each timed on its own with a roofline entry of its own.
+
+    Median of 20 CUDA-event timed calls, a 256 MiB write before each.  ``traffic`` is the DRAM
+    bytes per launch from the committed ncu record for this kernel source and workload, or null.
+    """
     import torch
 
     from scaled_dot_product_prefill_b200 import api
@@ -487,7 +513,7 @@ def other_workloads(dev, peaks):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     res = {}
     for name, spec in workloads.WORKLOADS.items():
-        if not isinstance(spec, workloads.PrefillSpec):
+        if not isinstance(spec, workloads.PrefillSpec) or name == PREFILL.name:
             continue
         pi = inputs.prefill_inputs(spec.B, spec.Hq, spec.Hkv, spec.Sq, spec.Skv, spec.D, spec.seed, spec.dtype)
         q, k, v = pi.q.to(dev), pi.k.to(dev), pi.v.to(dev)
@@ -497,9 +523,15 @@ def other_workloads(dev, peaks):
                        20, flush)
         fl = workloads.prefill_flops(spec)
         ach = fl / (ms * 1e-3) / 1e12
-        entry = {"ms": round(ms, 5), "TFLOP/s": round(ach, 2)}
+        entry = {"ms": round(ms, 5), "TFLOP/s": round(ach, 2), "flops": fl}
         if spec.dtype == "bf16":
-            entry["frac_of_bf16_peak"] = round(ach / float(peaks["bf16_tflops"]), 4)
+            peak = float(peaks["bf16_tflops"])
+            entry["roofline"] = {"bound": "tensor", "achieved": round(ach, 2), "peak": peak, "unit": "TFLOP/s",
+                                 "frac": round(ach / peak, 4),
+                                 "traffic": recorded_traffic("prefill_tc_kernel", name, "prefill_sm100.cu"),
+                                 "kernel": f"prefill_tc_kernel<{spec.D}, false>"}
+        else:
+            entry["traffic"] = recorded_traffic("prefill_f32_kernel", name, "prefill_f32.cu")
         res[name] = entry
         del q, k, v, out
     torch.cuda.empty_cache()

@@ -90,9 +90,10 @@ typedef struct CUstream_st* attn_stream_t;
 
 typedef enum {
   ATTN_OK = 0,
-  ATTN_ERR_INVALID_ARG = 1,   /* null pointer, negative size, Hq % Hkv != 0, misaligned pointer */
-  ATTN_ERR_UNSUPPORTED = 2,   /* valid but not implemented: head dim, page size, group size,
-                                 window without causal */
+  ATTN_ERR_INVALID_ARG = 1,   /* null pointer, negative size, Hq % Hkv != 0, misaligned pointer,
+                                 attention head dim other than 64 or 128 */
+  ATTN_ERR_UNSUPPORTED = 2,   /* valid but not implemented: page size, group size, window
+                                 without causal, an append row size */
   ATTN_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed (launch, descriptor, device query) */
   ATTN_ERR_TIMEOUT = 4,       /* a device-side wait gave up (reported by attn_device_status) */
   ATTN_ERR_BAD_PAGE = 5,      /* a page-table entry was outside [0, num_pages), or a sequence was
@@ -114,7 +115,7 @@ int attn_version(void);
  * q   : [B, Hq,  Sq,  D] bf16, contiguous (row-major, D innermost)
  * k, v: [B, Hkv, Skv, D] bf16, contiguous
  * out : [B, Hq,  Sq,  D] bf16, contiguous; must not alias q, k or v
- * D   : 64 or 128 (otherwise ATTN_ERR_UNSUPPORTED)
+ * D   : 64 or 128 (otherwise ATTN_ERR_INVALID_ARG)
  * scale : multiplier of q.k (1/sqrt(D) in the pages; passed explicitly)
  * causal: 0 or 1;  window: 0 = none, > 0 = sliding window (needs causal=1)
  *
@@ -122,8 +123,8 @@ int attn_version(void);
  * on tiles staged by TMA; the softmax is the online form (running row max
  * and sum, accumulator rescaled when the max grows) and P is rounded to
  * bf16 before P.V.  Key tiles that the mask hides entirely are skipped.
- * Errors: ATTN_ERR_INVALID_ARG for null/misaligned pointers or bad sizes,
- * ATTN_ERR_UNSUPPORTED for D not in {64,128} or window>0 without causal,
+ * Errors: ATTN_ERR_INVALID_ARG for null/misaligned pointers, bad sizes or D
+ * not in {64,128}, ATTN_ERR_UNSUPPORTED for window>0 without causal,
  * ATTN_ERR_CUDA if the tensor-map encoder or the launch fails.
  */
 attn_status_t attn_prefill(const void* q, const void* k, const void* v, void* out,

@@ -99,6 +99,12 @@ def attn_prefill(q, k, v, *, causal=False, window=0, scale=None, out=None, strea
 
 
 _COPY_STREAMS: dict = {}
+# Host tensors of attn_prefill_host calls whose copies may still be in flight, each
+# with an event recorded on the call's stream after its last copy.  The library
+# copies them with its own cudaMemcpyAsync calls, which torch's pinned-memory
+# allocator does not track, so a host tensor the caller drops could otherwise be
+# handed out again (and overwritten or read) while a copy still uses it.
+_HOST_IN_FLIGHT: list = []
 
 
 def _copy_streams(dev):
@@ -109,6 +115,11 @@ def _copy_streams(dev):
             pair = (torch.cuda.Stream(), torch.cuda.Stream())
         _COPY_STREAMS[dev] = pair
     return pair
+
+
+def _release_finished_host_calls():
+    while _HOST_IN_FLIGHT and _HOST_IN_FLIGHT[0][0].query():
+        _HOST_IN_FLIGHT.pop(0)
 
 
 def attn_prefill_host(q, k, v, *, causal=False, window=0, scale=None, out=None, chunks=0, device_buffers=None,
@@ -122,7 +133,8 @@ def attn_prefill_host(q, k, v, *, causal=False, window=0, scale=None, out=None, 
     tensors of the same shapes, allocated here if None.  `copy_streams` =
     (copy_in, copy_out) torch streams, "auto" for two per device, or None to
     copy on `stream`.  The returned host tensor is complete once `stream`
-    (default: the current stream) has completed.
+    (default: the current stream) has completed.  This binding keeps q, k,
+    v and out referenced until then, so the caller may drop them at once.
     """
     for t, name in ((q, "q"), (k, "k"), (v, "v")):
         if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
@@ -137,7 +149,8 @@ def attn_prefill_host(q, k, v, *, causal=False, window=0, scale=None, out=None, 
         raise ValueError("out must be a contiguous host tensor")
     _expect(out, "out", q.shape, torch.bfloat16)
     dev = torch.cuda.current_device()
-    if device_buffers is None:
+    own_buffers = device_buffers is None
+    if own_buffers:
         device_buffers = (torch.empty(q.shape, dtype=torch.bfloat16, device=dev),
                           torch.empty(k.shape, dtype=torch.bfloat16, device=dev),
                           torch.empty(v.shape, dtype=torch.bfloat16, device=dev),
@@ -149,18 +162,27 @@ def attn_prefill_host(q, k, v, *, causal=False, window=0, scale=None, out=None, 
     if copy_streams == "auto":
         copy_streams = _copy_streams(dev)
     cin, cout = copy_streams if copy_streams is not None else (None, None)
+    kernel_stream = torch.cuda.current_stream() if stream is None else stream
+    users = [cs for cs in (cin, cout) if cs is not None]
+    if own_buffers and kernel_stream != torch.cuda.current_stream():
+        users.append(kernel_stream)   # allocated on the current stream, used on another
     for t in (qd, kd, vd, od):   # the copy streams use the buffers too: keep them from early reuse
-        for cs in (cin, cout):
-            if cs is not None:
-                t.record_stream(cs)
+        for cs in users:
+            t.record_stream(cs)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
+    _release_finished_host_calls()
     _check("attn_prefill_host",
            _lib.load().attn_prefill_host(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(qd), _ptr(kd), _ptr(vd),
                                          _ptr(od), B, Hq, Hkv, Sq, Skv, D, float(scale), int(bool(causal)),
                                          int(window), int(chunks), _stream(stream),
                                          None if cin is None else ctypes_void(cin.cuda_stream),
                                          None if cout is None else ctypes_void(cout.cuda_stream)))
+    # the call joins its copy streams into `stream` before returning: an event
+    # recorded there completes after every copy that reads or writes the host tensors
+    done = torch.cuda.Event()
+    done.record(kernel_stream)
+    _HOST_IN_FLIGHT.append((done, (q, k, v, out)))
     return out
 
 

@@ -68,7 +68,7 @@ attn_status_t check_prefill(const void* q, const void* k, const void* v, const v
   // with no keys (Skv == 0) k and v are never read and may be null
   if (q == nullptr || out == nullptr || (Skv > 0 && (k == nullptr || v == nullptr))) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ATTN_ERR_INVALID_ARG;
-  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128) return ATTN_ERR_INVALID_ARG;
   if (window > 0 && !causal) return ATTN_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * Hq > 65535LL * 32768LL) return ATTN_ERR_UNSUPPORTED;
   return ATTN_OK;
@@ -164,7 +164,7 @@ attn_status_t attn_prefill_paged(const void* q, const void* k_pool, const void* 
       (reinterpret_cast<uintptr_t>(page_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u) ||
       (reinterpret_cast<uintptr_t>(lse) & 3u))
     return ATTN_ERR_INVALID_ARG;
-  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128) return ATTN_ERR_INVALID_ARG;
   if (window > 0 && !causal) return ATTN_ERR_UNSUPPORTED;
   if (page_size != 16 && page_size != 32 && page_size != 64 && page_size != 128 && page_size != 256)
     return ATTN_ERR_UNSUPPORTED;
@@ -293,7 +293,7 @@ attn_status_t decode_paged(const void* q, const void* k_pool, const void* v_pool
   if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out) ||
       (reinterpret_cast<uintptr_t>(page_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
     return ATTN_ERR_INVALID_ARG;
-  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128) return ATTN_ERR_INVALID_ARG;
   const int G = Hq / Hkv;
   if (G != 1 && G != 2 && G != 4 && G != 8) return ATTN_ERR_UNSUPPORTED;
   if (page_size % 16 != 0 || page_size > 256) return ATTN_ERR_UNSUPPORTED;

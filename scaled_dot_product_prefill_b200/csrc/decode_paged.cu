@@ -45,17 +45,9 @@ namespace {
 constexpr int kWarps = 4;       // warps per split CTA
 constexpr int kChunk = 16;      // tokens per chunk (one bulk copy per K and per V)
 constexpr float kTau = 8.0f;    // lazy-rescale threshold, log2 units
-// Ring depth per warp (16-token K+V chunks at D = 128; twice as many at D = 64)
-// and the CTAs per SM the register allocation aims for.
-#ifndef ATTN_DECODE_STAGES
-#define ATTN_DECODE_STAGES 2
-#endif
-#ifndef ATTN_DECODE_SPLIT
-#define ATTN_DECODE_SPLIT 512
-#endif
-#ifndef ATTN_DECODE_MINB
-#define ATTN_DECODE_MINB 3
-#endif
+constexpr int kStages = 2;      // ring depth per warp: 16-token K+V chunks at D = 128 (twice as many at D = 64)
+constexpr int kSplit = 512;     // keys per split when the batch fills the GPU
+constexpr int kMinBlocks = 3;   // CTAs per SM the register allocation aims for
 
 struct DecodeParams {
   const __nv_bfloat16* q;
@@ -152,7 +144,7 @@ struct Geo {
   static constexpr int TPL = 32 / R;              // tokens per warp-wide load
   static constexpr int NL = kChunk / TPL;         // loads per chunk per lane
   static constexpr int CHUNK_BYTES = kChunk * D * EB;
-  static constexpr int STAGES = ((D == 128) ? ATTN_DECODE_STAGES : 2 * ATTN_DECODE_STAGES) * (FP8 ? 2 : 1);
+  static constexpr int STAGES = ((D == 128) ? kStages : 2 * kStages) * (FP8 ? 2 : 1);
 };
 
 template <int D, int G, bool FP8>
@@ -167,7 +159,7 @@ struct SplitSmem {
 
 // Groups of 8 query heads hold twice the accumulators: 2 CTAs per SM leave them 255 registers.
 template <int D, int G, bool FP8>
-__global__ void __launch_bounds__(kWarps * 32, (G >= 8) ? 2 : ATTN_DECODE_MINB)
+__global__ void __launch_bounds__(kWarps * 32, (G >= 8) ? 2 : kMinBlocks)
     decode_split_kernel(const DecodeParams p) {
   using Gm = Geo<D, FP8>;
   constexpr int R = Gm::R, TPL = Gm::TPL, NL = Gm::NL, STAGES = Gm::STAGES;
@@ -515,10 +507,10 @@ DecodeGeometry decode_geometry(int N, int Hq, int D, int max_seq_len, int page_s
   (void)D;
   (void)page_size;
   DecodeGeometry g{};
-  // ATTN_DECODE_SPLIT keys per split (8 chunks per warp at 512), enough to
+  // kSplit keys per split (8 chunks per warp at 512), enough to
   // amortise the pipeline fill; shorter splits when the batch is too small
   // to fill the GPU.
-  int split = ATTN_DECODE_SPLIT;
+  int split = kSplit;
   const long long units = static_cast<long long>(N);
   while (split > 64 && units * ((max_seq_len + split - 1) / split) < 1024) split /= 2;
   g.split_tokens = split;

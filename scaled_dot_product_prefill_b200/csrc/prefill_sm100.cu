@@ -39,11 +39,7 @@
 // the softmax releases S_i as soon as it has loaded it, the MMA thread
 // computes S_i(j+1) while the exponentials of tile j run, and each P_i V_j
 // signals its own completion.  PAGED kernels read K/V through a page table
-// as page-sized TMA boxes.  Compile-time alternatives, measured and left
-// off: ATTN_D64_VARIANT=1 (two CTAs per SM over 64-key tiles),
-// ATTN_D128_VARIANT=2 (P in shared memory), ATTN_PREFILL_TURNS (the softmax
-// groups take turns at the exponentials), ATTN_EXP_EMU (part of the
-// exponentials on the FMA pipe).
+// as page-sized TMA boxes.
 #include <cmath>
 #include <cstdint>
 #include <cuda.h>
@@ -60,73 +56,38 @@ constexpr int BM = 128;          // query rows per tile
 constexpr int NQ = 2;            // query tiles per work item
 constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;
-#ifndef ATTN_PREFILL_TURNS
-#define ATTN_PREFILL_TURNS 0
-#endif
 constexpr float kTau = 8.0f;     // lazy-rescale threshold, log2 units
-// Of every 16 score pairs of a row, how many take exp2 on the FMA pipe
-// (exp2_fma2) instead of the MUFU unit, which is the bottleneck of the softmax.
-#ifndef ATTN_EXP_EMU
-#define ATTN_EXP_EMU 0
-#endif
-constexpr int kEmuPer16 = ATTN_EXP_EMU;
 
-// D=64 layouts: 0 = one CTA per SM, 128-key tiles and P buffers of their own
-// (below); 1 = two CTAs per SM, each with 64-key tiles, P over S and half of
-// tensor memory, so that an SM runs four softmax chains instead of two.
-#ifndef ATTN_D64_VARIANT
-#define ATTN_D64_VARIANT 0
-#endif
-// D=128 layouts: 0 = P written over S in tensor memory; 2 = P in shared memory
-// (a 3-slot K/V ring makes room), so that S_i(j+1) need not wait for P_i V(j).
-#ifndef ATTN_D128_VARIANT
-#define ATTN_D128_VARIANT 0
-#endif
-
-template <int D, int V = 0>
+template <int D>
 struct Cfg {
-  static_assert(V == 0 || (V == 1 && D == 64) || (V == 2 && D == 128), "layout variant");
-  static constexpr int BN = (V == 1) ? 64 : 128;      // keys per tile
-  static constexpr int MINB = (V == 1) ? 2 : 1;       // CTAs per SM
-  static constexpr uint32_t TMEM_COLS = (V == 1) ? 256 : 512;
-  // V = 0: 12 warps (3 warpgroups) and a register split (setmaxnreg works per
+  static constexpr int BN = 128;                      // keys per tile
+  // 12 warps (3 warpgroups) and a register split (setmaxnreg works per
   // warpgroup): the two softmax groups hold a 128-column score row each; the
   // producer group (TMA and MMA warps, two idle warps) gets the rest.
   // 128 * (2 * SOFTMAX_REGS + PRODUCER_REGS) must fit the launch allocation
   // (threads * registers per thread), which the host checks before the first
-  // launch.  V = 1: 10 warps (8 softmax, TMA, MMA) with about 100 registers
-  // each and no split.
-  static constexpr int THREADS = (V == 1) ? 320 : 384;
-  static constexpr bool SPLIT_REGS = (V == 0);
+  // launch.
+  static constexpr int THREADS = 384;
   static constexpr int SOFTMAX_REGS = 208;
   static constexpr int PRODUCER_REGS = 88;
   static constexpr int KATOMS = D / 64;               // 64-column (128-byte) swizzle atoms
   static constexpr int TILE_BYTES = BN * D * 2;       // one K or V tile
   static constexpr int Q_BYTES = BM * D * 2;          // one query tile
-  static constexpr int QBUF = (D == 128 || V == 1) ? 1 : 2;   // query buffers (items in flight)
-  static constexpr int STAGES = (D == 128) ? (V == 2 ? 3 : 4) : 6;   // ring slots; K and V tiles alternate
+  static constexpr int QBUF = (D == 128) ? 1 : 2;     // query buffers (items in flight)
+  static constexpr int STAGES = (D == 128) ? 4 : 6;   // ring slots; K and V tiles alternate
   // D = 64 leaves room in tensor memory for P buffers of their own (SEP_P):
   // S_i [128 i, +128), P_i [256 + 64 i, +64), O_i [384 + 64 i, +64).  The
-  // softmax then releases S_i as soon as it has loaded it, and S_i(j+1) is
-  // computed while the softmax of tile j is still running.  D = 128 has no
-  // room: P_i is written over the first 64 columns of S_i, O_i [256 + 128 i, +128).
-  static constexpr bool SEP_P = (D == 64 && V == 0) || V == 2;
-  static constexpr bool P_SMEM = (V == 2);            // P_i in shared memory, read by an SS-form P.V
-  static constexpr int P_BYTES = P_SMEM ? NQ * BM * BN * 2 : 0;
-  // O_i is rescaled after the exponentials (when its score registers are
-  // free) with separate P buffers, and in the small-register layout.
-  static constexpr bool LATE_RESCALE = SEP_P || V == 1;
-  // TURNS: the two softmax groups take turns at the exponentials, so that one
-  // group's exponentials run at the full MUFU rate while the other loads S,
-  // takes its row max and stores P (ATTN_PREFILL_TURNS: 0 never, 1 at D = 64,
-  // 2 always).
-  static constexpr bool TURNS = (ATTN_PREFILL_TURNS == 2) || (ATTN_PREFILL_TURNS == 1 && D == 64);
-  // V = 1: S_i [64 i, +64) with P_i over its first 32 columns, O_i [128 + 64 i, +64).
+  // softmax then releases S_i as soon as it has loaded it, S_i(j+1) is
+  // computed while the softmax of tile j is still running, and O_i is
+  // rescaled after the exponentials.  D = 128 has no room: P_i is written
+  // over the first 64 columns of S_i, O_i [256 + 128 i, +128).
+  static constexpr bool SEP_P = (D == 64);
+  static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t S_COL = 0;                // + BN * i
   static constexpr uint32_t P_COL = SEP_P ? 256 : 0;  // + P_STRIDE * i
   static constexpr uint32_t P_STRIDE = SEP_P ? 64 : BN;
-  static constexpr uint32_t O_COL = (SEP_P && !P_SMEM) ? 384 : NQ * BN;  // + D * i
-  static constexpr size_t SMEM = 1024 /*align*/ + QBUF * NQ * Q_BYTES + STAGES * TILE_BYTES + P_BYTES + 256;
+  static constexpr uint32_t O_COL = SEP_P ? 384 : NQ * BN;  // + D * i
+  static constexpr size_t SMEM = 1024 /*align*/ + QBUF * NQ * Q_BYTES + STAGES * TILE_BYTES + 256;
 };
 
 struct Params {
@@ -222,11 +183,11 @@ __device__ __forceinline__ bool tile_unmasked(const Params& p, int skv, int r0, 
 // PAGED selects K/V through a page table (chunked prefill over a paged cache)
 // instead of dense [B, Hkv, Skv, D] tensors; the dense kernel carries none of
 // the paged code.
-template <int D, bool PAGED, int V>
-__global__ void __launch_bounds__(Cfg<D, V>::THREADS, Cfg<D, V>::MINB)
+template <int D, bool PAGED>
+__global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_v, const Params p) {
-  using C = Cfg<D, V>;
+  using C = Cfg<D>;
   constexpr int BN = C::BN;
   constexpr int STAGES = C::STAGES, QBUF = C::QBUF;
   extern __shared__ uint8_t smem_raw[];
@@ -234,8 +195,7 @@ __global__ void __launch_bounds__(Cfg<D, V>::THREADS, Cfg<D, V>::MINB)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = smem;                                   // [QBUF][NQ][KATOMS][BM rows x 128 B]
   uint8_t* sRing = smem + QBUF * NQ * C::Q_BYTES;       // [STAGES][KATOMS][BN rows x 128 B]
-  uint8_t* sP = sRing + STAGES * C::TILE_BYTES;         // P_SMEM: [NQ][BN / 64][BM rows x 128 B]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + C::P_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sRing + STAGES * C::TILE_BYTES);
   uint64_t* q_full = bars;                              // QBUF
   uint64_t* q_empty = q_full + QBUF;                    // QBUF
   uint64_t* full = q_empty + QBUF;                      // STAGES
@@ -245,8 +205,7 @@ __global__ void __launch_bounds__(Cfg<D, V>::THREADS, Cfg<D, V>::MINB)
   uint64_t* o_done = p_ready + NQ;                      // NQ: O_i final (SEP_P: each P_i V done)
   uint64_t* s_free = o_done + NQ;                       // NQ: S_i loaded by the softmax (SEP_P)
   uint64_t* drain = s_free + NQ;                        // 1
-  uint64_t* turn = drain + 1;                           // NQ: group i may run its exponentials (TURNS)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(turn + NQ);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -266,7 +225,6 @@ __global__ void __launch_bounds__(Cfg<D, V>::THREADS, Cfg<D, V>::MINB)
       mbar_init(&p_ready[i], 4 * 32);
       mbar_init(&o_done[i], 1);
       mbar_init(&s_free[i], 4 * 32);
-      mbar_init(&turn[i], 4 * 32);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -283,7 +241,7 @@ __global__ void __launch_bounds__(Cfg<D, V>::THREADS, Cfg<D, V>::MINB)
 
   if (warp >= 8) {
    // ------------------------------------------------------------ producer warpgroup
-   if constexpr (C::SPLIT_REGS) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::PRODUCER_REGS));
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::PRODUCER_REGS));
    if (warp == kTmaWarp) {
     // ------------------------------------------------------------ TMA producer
     // Dense: one thread.  Paged: the whole warp, so that the page-table
@@ -382,7 +340,6 @@ __global__ void __launch_bounds__(Cfg<D, V>::THREADS, Cfg<D, V>::MINB)
       const uint32_t q_lo0 = sw128_desc_lo(smem_u32(sQ), 16);
       const uint32_t k_lo0 = sw128_desc_lo(smem_u32(sRing), 16);
       const uint32_t v_lo0 = sw128_desc_lo(smem_u32(sRing), BN * 128);
-      const uint32_t p_lo0 = sw128_desc_lo(smem_u32(sP), 16);   // P_SMEM only
       int n = 0, qn = 0;
       int ts[NQ] = {0, 0};
       bool ok = true;
@@ -477,21 +434,11 @@ __global__ void __launch_bounds__(Cfg<D, V>::THREADS, Cfg<D, V>::MINB)
               const uint32_t o_tmem = tmem + C::O_COL + D * i;
               const uint32_t vb_lo = v_lo0 + ((stV * C::TILE_BYTES) >> 4);
               const uint32_t acc0 = (j > it.lo[i]) ? 1u : 0u;
-              if constexpr (C::P_SMEM) {   // A = P_i, K-major in shared memory like a Q tile
-                const uint32_t pa_lo = p_lo0 + ((i * BM * BN * 2) >> 4);
+              const uint32_t p_tmem = tmem + C::P_COL + C::P_STRIDE * i;
 #pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
-                  const uint32_t koff = ((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4;
-                  mma_ss(o_tmem, desc64(pa_lo + koff, kHi), desc64(vb_lo + ((kk * 16 * 128) >> 4), kHi), idesc_pv,
-                         kk > 0 ? 1u : acc0);
-                }
-              } else {
-                const uint32_t p_tmem = tmem + C::P_COL + C::P_STRIDE * i;
-#pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk)
-                  mma_ts(o_tmem, p_tmem + kk * 8, desc64(vb_lo + ((kk * 16 * 128) >> 4), kHi), idesc_pv,
-                         kk > 0 ? 1u : acc0);
-              }
+              for (int kk = 0; kk < BN / 16; ++kk)
+                mma_ts(o_tmem, p_tmem + kk * 8, desc64(vb_lo + ((kk * 16 * 128) >> 4), kHi), idesc_pv,
+                       kk > 0 ? 1u : acc0);
               mma_commit(&o_done[i]);   // P_i free again, O_i current
             }
             if (!ok) break;
@@ -567,7 +514,7 @@ __global__ void __launch_bounds__(Cfg<D, V>::THREADS, Cfg<D, V>::MINB)
    }
   } else {
     // ------------------------------------------------------------ softmax groups
-    if constexpr (C::SPLIT_REGS) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::SOFTMAX_REGS));
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::SOFTMAX_REGS));
     const int i = warp >> 2;                 // query tile
     const int wq = warp & 3;                 // lane quarter of tensor memory
     const int rl = wq * 32 + lane;           // row within the tile
@@ -578,20 +525,6 @@ __global__ void __launch_bounds__(Cfg<D, V>::THREADS, Cfg<D, V>::MINB)
     const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
     int t = 0, oc = 0;
     int pv = 0;   // SEP_P: P_i V products of this tile completed and waited for
-    // Turns at the exponentials (TURNS): group 0 goes first; each group waits
-    // for its turn, runs its exponentials and hands the turn over.  Both groups
-    // take the same number of turns per item: the one with fewer key tiles
-    // takes empty turns first.  Group 1 opens group 0's first turn.
-    int tk = 0;   // turns this group has waited for
-    if constexpr (C::TURNS) {
-      if (i == 1) mbar_arrive(&turn[0]);
-    }
-    auto take_turn = [&]() -> bool {
-      const bool r = mbar_wait(&turn[i], tk & 1, abort_flag, p.err);
-      ++tk;
-      return __all_sync(0xffffffffu, r);
-    };
-    auto pass_turn = [&]() { mbar_arrive(&turn[1 - i]); };
     // O_i *= alpha (every row of the warp takes part when any row needs it)
     auto rescale_o = [&](bool later_tile, float alpha) {
       if (!__any_sync(0xffffffffu, later_tile && alpha != 1.f)) return;
@@ -619,15 +552,6 @@ __global__ void __launch_bounds__(Cfg<D, V>::THREADS, Cfg<D, V>::MINB)
       const Item it = make_item<BN, PAGED>(p, k);
       const int my_lo = (i == 0) ? it.lo[0] : it.lo[1];
       const int my_hi = (i == 0) ? it.hi[0] : it.hi[1];
-      if constexpr (C::TURNS) {
-        const int n_mine = max(0, my_hi - my_lo);
-        const int n_other = (i == 0) ? max(0, it.hi[1] - it.lo[1]) : max(0, it.hi[0] - it.lo[0]);
-        for (int e = n_mine; e < n_other && ok; ++e) {
-          ok = take_turn();
-          if (ok) pass_turn();
-        }
-        if (!ok) break;
-      }
       const int r0 = it.q_row0 + BM * i;
       const int r = r0 + rl;                 // query row of this thread
       const bool store = r < p.Sq;
@@ -684,10 +608,7 @@ __global__ void __launch_bounds__(Cfg<D, V>::THREADS, Cfg<D, V>::MINB)
           l *= alpha;
           m_ref = m_tile;
         }
-        if constexpr (!C::LATE_RESCALE) rescale_o(j > my_lo, alpha);   // O_i is current: S_i(j) covers P_i V(j-1)
-        if constexpr (C::TURNS) {
-          if (!(ok = take_turn())) break;
-        }
+        if constexpr (!C::SEP_P) rescale_o(j > my_lo, alpha);   // O_i is current: S_i(j) covers P_i V(j-1)
         const float mb = (m_ref == -INFINITY) ? 0.f : m_ref;
         const uint64_t nm2 = f2_pack(-mb, -mb);
         uint32_t pk[BN / 2];
@@ -697,15 +618,9 @@ __global__ void __launch_bounds__(Cfg<D, V>::THREADS, Cfg<D, V>::MINB)
 #pragma unroll
         for (int c = 0; c < BN; c += 2) {
           const uint64_t x2 = f2_fma(f2_pack(s[c], s[c + 1]), c2, nm2);
-          float p0, p1;
-          if ((c / 2) % 16 < kEmuPer16) {
-            f2_unpack(exp2_fma2(x2), p0, p1);
-          } else {
-            float x0, x1;
-            f2_unpack(x2, x0, x1);
-            p0 = ex2(x0);
-            p1 = ex2(x1);
-          }
+          float x0, x1;
+          f2_unpack(x2, x0, x1);
+          const float p0 = ex2(x0), p1 = ex2(x1);
           sum2[(c / 2) % 4] = f2_add(sum2[(c / 2) % 4], f2_pack(p0, p1));
           pk[c / 2] = pack_bf16x2(p0, p1);
         }
@@ -713,7 +628,6 @@ __global__ void __launch_bounds__(Cfg<D, V>::THREADS, Cfg<D, V>::MINB)
         f2_unpack(f2_add(sum2[0], sum2[1]), s0, s1);
         f2_unpack(f2_add(sum2[2], sum2[3]), s2, s3);
         l += (s0 + s1) + (s2 + s3);
-        if constexpr (C::TURNS) pass_turn();
         // The exponentials above need nothing from tensor memory; only now must
         // P_i(j-1) V be complete: before O_i is rescaled and (separate P) before
         // P_i is rewritten.  Waiting here hides that product behind them.
@@ -728,24 +642,10 @@ __global__ void __launch_bounds__(Cfg<D, V>::THREADS, Cfg<D, V>::MINB)
             tc_fence_after();
           }
         }
-        if constexpr (C::LATE_RESCALE) rescale_o(j > my_lo, alpha);
-        if constexpr (C::P_SMEM) {
-          // row rl of P_i in the 128-byte-swizzled K-major layout the MMA reads:
-          // 16-byte chunk c of a 128-byte row lands at chunk c ^ (row % 8)
-          const uint32_t prow = smem_u32(sP) + i * (BM * BN * 2) + rl * 128;
+        if constexpr (C::SEP_P) rescale_o(j > my_lo, alpha);
 #pragma unroll
-          for (int ch = 0; ch < BN / 8; ++ch) {
-            const uint32_t addr = prow + (ch >> 3) * (BM * 128) + (((ch & 7) ^ (rl & 7)) << 4);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * ch]),
-                         "r"(pk[4 * ch + 1]), "r"(pk[4 * ch + 2]), "r"(pk[4 * ch + 3])
-                         : "memory");
-          }
-          fence_proxy_async_smem();   // the MMA reads P through the async proxy
-        } else {
-#pragma unroll
-          for (int c = 0; c < BN / 64; ++c) tmem_st32(p_tmem + 32 * c, pk + 32 * c);
-          tmem_wait_st();
-        }
+        for (int c = 0; c < BN / 64; ++c) tmem_st32(p_tmem + 32 * c, pk + 32 * c);
+        tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&p_ready[i]);
       }
@@ -763,8 +663,7 @@ __global__ void __launch_bounds__(Cfg<D, V>::THREADS, Cfg<D, V>::MINB)
         break;
       }
       tc_fence_after();
-      // a row with no visible key is 0 (the FMA-pipe exp2 maps masked scores
-      // to about 2^-126 instead of exactly 0)
+      // a row with no visible key is 0 (and its lse -inf)
       const bool has_keys = key_hi >= max(key_lo, 0);
       const float inv = (has_keys && l > 0.f) ? 1.f / l : 0.f;
       if (p.lse != nullptr && store)   // log(sum_j exp(s_ij * scale)) = (m + log2 l) * ln 2
@@ -851,37 +750,37 @@ int sm_count() {
 // block's own registers cover the request, so a build whose launch
 // allocation could not is refused).  Done once per device; later calls skip
 // the runtime queries, which cost more host time than the launch itself.
-template <int D, bool PAGED, int V>
+template <int D, bool PAGED>
 cudaError_t prepare_kernel() {
-  using C = Cfg<D, V>;
+  using C = Cfg<D>;
   constexpr int kMaxDevices = 64;
   static int ready[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   if (__atomic_load_n(&ready[dev], __ATOMIC_ACQUIRE) == 1) return cudaSuccess;
-  auto kern = prefill_tc_kernel<D, PAGED, V>;
+  auto kern = prefill_tc_kernel<D, PAGED>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM));
   if (e != cudaSuccess) return e;
   cudaFuncAttributes fa{};
   e = cudaFuncGetAttributes(&fa, kern);
   if (e != cudaSuccess) return e;
-  if (C::SPLIT_REGS && fa.numRegs * C::THREADS < 128 * (2 * C::SOFTMAX_REGS + C::PRODUCER_REGS))
+  if (fa.numRegs * C::THREADS < 128 * (2 * C::SOFTMAX_REGS + C::PRODUCER_REGS))
     return cudaErrorInvalidConfiguration;
   __atomic_store_n(&ready[dev], 1, __ATOMIC_RELEASE);
   return cudaSuccess;
 }
 
-template <int D, bool PAGED, int V>
+template <int D, bool PAGED>
 cudaError_t launch_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const Params& p,
                      cudaStream_t stream) {
-  using C = Cfg<D, V>;
-  auto kern = prefill_tc_kernel<D, PAGED, V>;
+  using C = Cfg<D>;
+  auto kern = prefill_tc_kernel<D, PAGED>;
   const size_t smem = C::SMEM;
-  cudaError_t e = prepare_kernel<D, PAGED, V>();
+  cudaError_t e = prepare_kernel<D, PAGED>();
   if (e != cudaSuccess) return e;
   const int sms = sm_count();
   if (sms <= 0) return cudaErrorInvalidDevice;
-  const unsigned grid = static_cast<unsigned>(min(p.n_items, sms * C::MINB));
+  const unsigned grid = static_cast<unsigned>(min(p.n_items, sms));
   kern<<<grid, C::THREADS, smem, stream>>>(mq, mk, mv, p);
   return cudaGetLastError();
 }
@@ -891,8 +790,7 @@ cudaError_t launch_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
 cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
                               int Hkv, int Sq, int Skv, int D, float scale, int causal, int window, unsigned int* err,
                               cudaStream_t stream) {
-  constexpr int V64 = ATTN_D64_VARIANT;
-  const int bn = (D == 64) ? Cfg<64, V64>::BN : Cfg<128, ATTN_D128_VARIANT>::BN;
+  const int bn = (D == 64) ? Cfg<64>::BN : Cfg<128>::BN;
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, q, D, Sq, B * Hq) || !make_map(&mk, k, D, Skv, B * Hkv, bn) ||
       !make_map(&mv, v, D, Skv, B * Hkv, bn))
@@ -913,16 +811,14 @@ cudaError_t launch_prefill_tc(const void* q, const void* k, const void* v, void*
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
   p.err = err;
-  return D == 64 ? launch_d<64, false, V64>(mq, mk, mv, p, stream)
-                 : launch_d<128, false, ATTN_D128_VARIANT>(mq, mk, mv, p, stream);
+  return D == 64 ? launch_d<64, false>(mq, mk, mv, p, stream) : launch_d<128, false>(mq, mk, mv, p, stream);
 }
 
 cudaError_t launch_prefill_tc_paged(const void* q, const void* k_pool, const void* v_pool, const int32_t* page_table,
                                     const int32_t* seq_lens, int page_size, int B, int Hq, int Hkv, int Sq, int D,
                                     int num_pages, int max_pages, int max_seq_len, float scale, int causal,
                                     int window, void* out, float* lse, unsigned int* err, cudaStream_t stream) {
-  constexpr int V64 = ATTN_D64_VARIANT;
-  const int bn = (D == 64) ? Cfg<64, V64>::BN : Cfg<128, ATTN_D128_VARIANT>::BN;
+  const int bn = (D == 64) ? Cfg<64>::BN : Cfg<128>::BN;
   const int box_rows = page_size < bn ? page_size : bn;
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, q, D, Sq, B * Hq) || !make_map(&mk, k_pool, D, page_size, num_pages * Hkv, box_rows) ||
@@ -950,8 +846,7 @@ cudaError_t launch_prefill_tc_paged(const void* q, const void* k_pool, const voi
   p.box_rows = box_rows;
   p.max_pages = max_pages;
   p.num_pages = num_pages;
-  return D == 64 ? launch_d<64, true, V64>(mq, mk, mv, p, stream)
-                 : launch_d<128, true, ATTN_D128_VARIANT>(mq, mk, mv, p, stream);
+  return D == 64 ? launch_d<64, true>(mq, mk, mv, p, stream) : launch_d<128, true>(mq, mk, mv, p, stream);
 }
 
 }  // namespace attn

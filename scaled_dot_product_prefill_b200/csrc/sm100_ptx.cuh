@@ -303,35 +303,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// 2^x for a pair of x, on the FMA and integer pipes instead of the MUFU unit.
-// Cody-Waite range reduction: x = n + f with n = round(x) (read from the low
-// bits of x + 1.5*2^23) and f in [-1/2, 1/2]; 2^f by a degree-3 polynomial
-// whose coefficients minimise the maximum relative error on [-1/2, 1/2]
-// (Lawson's iteratively reweighted least-squares algorithm; fitted by
-// csrc/fit_exp2_poly.py, max relative error 7.5e-5, below bf16's 2^-9);
-// 2^n is applied by adding n to the exponent field.  x is clamped below at
-// -126 so that the exponent field never underflows: results below 2^-126
-// come out as about 2^-126 or a denormal, never as garbage.
-__device__ __forceinline__ uint64_t exp2_fma2(uint64_t x2) {
-  constexpr float kC0 = 0.9999280571937561f, kC1 = 0.6932609677314758f;
-  constexpr float kC2 = 0.2426111400127411f, kC3 = 0.0551716685295105f;
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  float x0, x1;
-  f2_unpack(x2, x0, x1);
-  x2 = f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
-  const uint64_t t2 = f2_add(x2, f2_pack(kRound, kRound));
-  const uint64_t f = f2_sub(x2, f2_sub(t2, f2_pack(kRound, kRound)));
-  uint64_t p = f2_fma(f2_pack(kC3, kC3), f, f2_pack(kC2, kC2));
-  p = f2_fma(p, f, f2_pack(kC1, kC1));
-  p = f2_fma(p, f, f2_pack(kC0, kC0));
-  float p0, p1, t0, t1;
-  f2_unpack(p, p0, p1);
-  f2_unpack(t2, t0, t1);
-  p0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-  p1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-  return f2_pack(p0, p1);
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half), .y = hi
   return *reinterpret_cast<uint32_t*>(&v);

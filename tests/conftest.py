@@ -40,7 +40,20 @@ BF16_MAX_ABS, BF16_MEAN_ABS = 2e-2, 2e-3
 F32_MAX_ABS = 1e-4
 
 
-def assert_parity(got, ref, dtype="bf16", what=""):
+# (what, elements, max-abs, mean-abs) of the comparisons made with report=True, printed at
+# the end of the session (also under -q) so that the log carries the measured errors.
+PARITY_REPORT = []
+
+
+def pytest_terminal_summary(terminalreporter):
+    if not PARITY_REPORT:
+        return
+    terminalreporter.write_sep("-", "parity against the float64 oracle (whole outputs)")
+    for what, n, mx, mean in PARITY_REPORT:
+        terminalreporter.write_line(f"{what}: {n} elements, max-abs {mx:.3e}, mean-abs {mean:.3e}")
+
+
+def assert_parity(got, ref, dtype="bf16", what="", report=False):
     """Element-by-element comparison of a GPU result with the float64 oracle."""
     import numpy as np
 
@@ -50,6 +63,8 @@ def assert_parity(got, ref, dtype="bf16", what=""):
     assert np.all(np.isfinite(g)), f"{what}: non-finite output"
     err = np.abs(g - r)
     mx, mean = float(err.max()) if err.size else 0.0, float(err.mean()) if err.size else 0.0
+    if report:
+        PARITY_REPORT.append((what, int(err.size), mx, mean))
     if dtype == "bf16":
         assert mx <= BF16_MAX_ABS and mean <= BF16_MEAN_ABS, f"{what}: max-abs {mx:.3e} mean-abs {mean:.3e}"
     else:

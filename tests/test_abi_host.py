@@ -75,7 +75,7 @@ def test_prefill_argument_validation(fn):
     assert prefill(lib, fn, scale=float("nan")) == 1
     assert prefill(lib, fn, causal=2) == 1
     assert prefill(lib, fn, window=-3) == 1
-    assert prefill(lib, fn, D=96) == 2                  # head dim not implemented
+    assert prefill(lib, fn, D=96) == 1                  # head dim outside {64, 128}
     assert prefill(lib, fn, causal=0, window=16) == 2   # a window is a causal look-back
     # empty problems are no-ops, even with null pointers
     assert prefill(lib, fn, q=None, k=None, v=None, o=None, B=0) == 0
@@ -95,7 +95,7 @@ def test_decode_argument_validation():
     assert decode(lib, Hq=8, Hkv=3) == 1
     assert decode(lib, kp=MISALIGNED) == 1
     assert decode(lib, scale=-1.0) == 1
-    assert decode(lib, D=96) == 2
+    assert decode(lib, D=96) == 1
     assert decode(lib, Hq=24, Hkv=2) == 2               # group of 12
     assert decode(lib, page=8) == 2
     assert decode(lib, ws=None) == 6
@@ -132,7 +132,7 @@ def test_prefill_lse_argument_validation(fn):
                                               kw.get("D", 64), 0.125, 1, 0, None)
     assert call(None) == 1                        # the lse output is required
     assert call(ctypes.c_void_p(0x10002)) == 1    # misaligned lse
-    assert call(FAKE, D=96) == 2
+    assert call(FAKE, D=96) == 1
     assert call(None, B=0) == 0                   # empty problem
 
 
@@ -147,7 +147,7 @@ def test_paged_prefill_argument_validation():
     assert call(lse=ctypes.c_void_p(0x10002)) == 1
     assert call(page=8) == 2
     assert call(page=48) == 2
-    assert call(D=96) == 2
+    assert call(D=96) == 1
     assert call(causal=0, window=16) == 2
 
 
@@ -203,7 +203,7 @@ def test_fp8_decode_argument_validation():
     assert call(ks=float("nan")) == 1
     assert call(kp=None) == 1
     assert call(kp=MISALIGNED) == 1
-    assert call(D=96) == 2
+    assert call(D=96) == 1
     assert call(Hq=24, Hkv=2) == 2
     assert call(ws=None) == 6
 
@@ -249,5 +249,5 @@ def test_host_prefill_argument_validation():
     assert call(qd=MISALIGNED) == 1
     assert call(chunks=-1) == 1
     assert call(chunks=5) == 1                   # more pieces than (batch, kv head) pairs (2 x 2)
-    assert call(D=96) == 2
+    assert call(D=96) == 1
     assert call(B=0, qh=None, oh=None, qd=None, od=None) == 0   # empty problem

@@ -48,7 +48,7 @@ def test_paged_decode_workload_full():
     assert api.attn_device_status(clear=True) == 0
     ref = sdpa.decode_paged(p.q, p.k_pool, p.v_pool, p.page_table, p.seq_lens, spec.page_size, spec.scale,
                             spec.window)
-    assert_parity(out, ref, "bf16", spec.name)
+    assert_parity(out, ref, "bf16", spec.name, report=True)
 
 
 def test_page_permutation_and_poison_do_not_change_the_result():

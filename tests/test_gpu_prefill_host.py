@@ -71,11 +71,35 @@ def test_back_to_back_calls_reusing_device_buffers():
     B, Hq, Hkv, Sq, Skv, D = shape
     bufs = tuple(torch.empty(s, dtype=torch.bfloat16, device="cuda")
                  for s in ((B, Hq, Sq, D), (B, Hkv, Skv, D), (B, Hkv, Skv, D), (B, Hq, Sq, D)))
-    outs, refs = [], []
+    outs, refs, hosts = [], [], []
     for seed in (11, 12, 13):
         inp, qh, kh, vh = host_inputs(shape, seed=seed)
         outs.append(api.attn_prefill_host(qh, kh, vh, causal=True, chunks=6, device_buffers=bufs))
         refs.append(inp)
+        hosts.append((qh, kh, vh))   # held here until the copies are known to be done
+    torch.cuda.synchronize()
+    for out, inp in zip(outs, refs):
+        assert torch.equal(out, device_reference(inp, True, 0))
+
+
+def test_dropped_host_inputs_are_kept_until_the_copies_finish():
+    """The binding holds the host tensors until the call's stream has passed it.
+
+    The caller drops its pinned inputs right after each call and fills freshly
+    pinned buffers of the same size with NaN: had a dropped block been handed
+    out again while its copy was still queued, NaN would reach the output.
+    """
+    shape = (4, 8, 8, 512, 512, 64)
+    refs, outs = [], []
+    blocker = torch.empty(64 << 20, dtype=torch.uint8, device="cuda")
+    for seed in (21, 22, 23, 24):
+        blocker.zero_()   # keeps the stream busy, so that the copies are still queued below
+        inp, qh, kh, vh = host_inputs(shape, seed=seed)
+        outs.append(api.attn_prefill_host(qh, kh, vh, causal=True, chunks=4))
+        refs.append(inp)
+        del qh, kh, vh
+        junk = [torch.full(t.shape, float("nan"), dtype=torch.bfloat16).pin_memory() for t in (inp.q, inp.k, inp.v)]
+        del junk
     torch.cuda.synchronize()
     for out, inp in zip(outs, refs):
         assert torch.equal(out, device_reference(inp, True, 0))
