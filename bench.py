@@ -323,6 +323,33 @@ def run_ours(args, rank, world, local_rank):
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
     d2h = hout.numel() * hout.element_size()
 
+    # ---- the decode half end to end: the step's query and new key/value from pinned host memory, appended
+    # to the resident cache, decoded, and the output read back, in one attn_decode_step_host call
+    gen = np.random.default_rng(rank)
+    dq_h = pd.q.pin_memory()
+    kn_h = torch.from_numpy(gen.standard_normal((dspec.N, dspec.Hkv, 1, dspec.D), dtype=np.float32)).to(
+        torch.bfloat16).pin_memory()
+    vn_h = torch.from_numpy(gen.standard_normal((dspec.N, dspec.Hkv, 1, dspec.D), dtype=np.float32)).to(
+        torch.bfloat16).pin_memory()
+    dout_h = torch.empty_like(pd.q).pin_memory()
+    dbufs = (torch.empty_like(dq), torch.empty(kn_h.shape, dtype=torch.bfloat16, device=dev),
+             torch.empty(vn_h.shape, dtype=torch.bfloat16, device=dev), torch.empty_like(dq))
+    d_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(e_steps)]
+    for i in range(e_steps + 3):
+        ev = d_ev[i - 3] if i >= 3 else None
+        if ev:
+            ev[0].record()
+        api.attn_decode_step_host(dq_h, kn_h, vn_h, kp, vp, pt, sl, max_seq_len=msl, scale=dspec.scale,
+                                  window=dspec.window, out=dout_h, device_buffers=dbufs, workspace=ws)
+        if ev:
+            ev[1].record()
+    torch.cuda.synchronize()
+    assert api.attn_device_status(clear=True) == 0
+    e2e_dec_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in d_ev]))
+    (e2e_dec_ms,) = max_over_ranks([e2e_dec_ms], dist, dev)
+    h2d_dec = sum(t.numel() * t.element_size() for t in (dq_h, kn_h, vn_h))
+    d2h_dec = dout_h.numel() * dout_h.element_size()
+
     # ---- the prefill replayed from a CUDA graph: the same kernel without the host launch path
     graph_ms = None
     if rank == 0 and not args.no_extra:
@@ -377,6 +404,11 @@ def run_ours(args, rank, world, local_rank):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms": round(e2e_ms, 5),
                     "path": "attn_prefill_host: pinned host q/k/v -> device -> kernels -> pinned host out, "
                             "in pieces whose copies overlap the kernels"},
+            "e2e_decode": {"value": round(job_rate(d_bytes, world, e2e_dec_ms) / 1e9, 1), "unit": "GB/s",
+                           "h2d_bytes_per_step": h2d_dec, "d2h_bytes_per_step": d2h_dec,
+                           "ms": round(e2e_dec_ms, 5),
+                           "path": "attn_decode_step_host: pinned host q and new k/v -> device -> append -> "
+                                   "decode -> pinned host out"},
             "gpu_launches": 3 * args.steps,
             "clocks": clk.summary(),
             "workloads": extra,

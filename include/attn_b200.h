@@ -36,6 +36,8 @@
  *                                     in the paged cache.
  *   attn_prefill_host                 the prefill from and to host memory, its
  *                                     copies overlapped with the kernels.
+ *   attn_decode_step_host             one decode step from and to host memory:
+ *                                     copy in, append, decode, copy out.
  *   attn_decode_paged_fp8             the decode over a cache of 8-bit E4M3
  *                                     codes (not on the pages: a storage
  *                                     variant).
@@ -279,6 +281,42 @@ attn_status_t attn_decode_paged(const void* q, const void* k_pool, const void* v
                                 float scale, int window,
                                 void* workspace, size_t workspace_bytes,
                                 void* out, attn_stream_t stream);
+
+/*
+ * attn_decode_step_host -- one serving decode step whose per-step inputs and
+ * output live in host memory ("Taking LLMs apart (2)", section "KV cache":
+ * each step stores the new token's key and value in the cache, then attends
+ * over the whole cache; "Attention From Scratch" README, section "Paged KV
+ * Cache": the cache is a shared pool of pages).  On `stream`, in order:
+ *   1. q_host -> q_dev, k_new_host -> k_new_dev, v_new_host -> v_new_dev;
+ *   2. attn_kv_append of the new token (S_new = 1) at position
+ *      seq_lens[b] - 1 of every sequence (seq_lens already counts it);
+ *   3. attn_decode_paged over the pools into out_dev;
+ *   4. out_dev -> out_host.
+ * The cache (pools, page_table, seq_lens, workspace) stays on the device:
+ * it is state, not per-step input.
+ *
+ * q_host, out_host : [N, Hq, D] bf16 host buffers; k_new_host, v_new_host :
+ *     [N, Hkv, 1, D] bf16.  Page-locked memory is needed for the copies to
+ *     run asynchronously; the host must not touch out_host, nor change the
+ *     inputs, until `stream` has completed.
+ * q_dev, out_dev : [N, Hq, D] bf16 device buffers; k_new_dev, v_new_dev :
+ *     [N, Hkv, 1, D]; owned by the caller, 16-byte aligned, overwritten.
+ * Other arguments : as attn_decode_paged (the pools are written by the
+ *     append, so they are not const here).
+ * Errors: as attn_kv_append and attn_decode_paged; ATTN_ERR_INVALID_ARG for a
+ * null host or device buffer; ATTN_ERR_CUDA if a copy or launch fails (work
+ * enqueued before the failure stays enqueued).
+ */
+attn_status_t attn_decode_step_host(const void* q_host, const void* k_new_host, const void* v_new_host,
+                                    void* out_host, void* q_dev, void* k_new_dev, void* v_new_dev,
+                                    void* out_dev, void* k_pool, void* v_pool,
+                                    const int32_t* page_table, const int32_t* seq_lens,
+                                    int page_size, int N, int Hq, int Hkv, int D,
+                                    int num_pages, int max_pages, int max_seq_len,
+                                    float scale, int window,
+                                    void* workspace, size_t workspace_bytes,
+                                    attn_stream_t stream);
 
 /*
  * attn_decode_paged_noalloc -- attn_decode_paged for callers that cannot

@@ -26,6 +26,7 @@ PROTOTYPES = {
     "attn_decode_paged": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 8 + [_c_float, _c_int, _vp, _c_size,
                                                                           _vp, _vp]),
     "attn_decode_paged_fp8": (_c_int, [_vp] * 5 + [_c_int] * 8 + [_c_float] * 3 + [_c_int, _vp, _c_size, _vp, _vp]),
+    "attn_decode_step_host": (_c_int, [_vp] * 12 + [_c_int] * 8 + [_c_float, _c_int, _vp, _c_size, _vp]),
     "attn_decode_paged_noalloc": (_c_int, [_vp, _vp, _vp, _vp, _vp] + [_c_int] * 8 + [_c_float, _c_int, _vp, _vp]),
     "attn_decode_paged_workspace_size": (_c_size, [_c_int] * 5),
     "attn_device_status": (_c_int, [_c_int]),

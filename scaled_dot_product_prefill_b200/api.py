@@ -15,6 +15,7 @@ from ._lib import AttnError
 
 __all__ = ["attn_prefill", "attn_prefill_f32", "attn_prefill_lse", "attn_prefill_f32_lse",
            "attn_prefill_paged", "attn_prefill_host", "attn_decode_paged", "attn_decode_paged_noalloc",
+           "attn_decode_step_host",
            "attn_decode_paged_workspace_size", "attn_decode_paged_fp8", "attn_kv_append", "attn_kv_append_fp8",
            "PagePool",
            "attn_device_status", "attn_selftest_wait_timeout", "attn_status_string", "attn_version", "AttnError"]
@@ -320,6 +321,66 @@ def attn_decode_paged_fp8(q, k_pool, v_pool, page_table, seq_lens, *, max_seq_le
         _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(page_table), _ptr(seq_lens), page_size, N, Hq, Hkv, D,
         num_pages, max_pages, int(max_seq_len), float(scale), float(k_scale), float(v_scale), int(window),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(out), _stream(stream)))
+    return out
+
+
+def attn_decode_step_host(q, k_new, v_new, k_pool, v_pool, page_table, seq_lens, *, max_seq_len, scale=None,
+                          window=0, out=None, device_buffers=None, workspace=None, stream=None):
+    """One decode step whose inputs and output are host tensors: copy in, append, decode, copy out.
+
+    q [N,Hq,D] and the new token's k_new/v_new [N,Hkv,1,D] are bf16 host
+    tensors (page-locked for asynchronous copies); the pools, page_table and
+    seq_lens (already counting the new token) are the device-resident cache.
+    `device_buffers` = (q_dev, k_new_dev, v_new_dev, out_dev), allocated here
+    if None.  The returned host tensor is complete once `stream` (default: the
+    current stream) has completed; this binding keeps the host tensors
+    referenced until then.
+    """
+    for t, name in ((q, "q"), (k_new, "k_new"), (v_new, "v_new")):
+        if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 host tensor")
+    N, Hq, D = q.shape
+    num_pages, Hkv, page_size, _ = k_pool.shape
+    _expect(k_new, "k_new", (N, Hkv, 1, D), torch.bfloat16)
+    _expect(v_new, "v_new", (N, Hkv, 1, D), torch.bfloat16)
+    _expect(k_pool, "k_pool", (num_pages, Hkv, page_size, D), torch.bfloat16)
+    _expect(v_pool, "v_pool", (num_pages, Hkv, page_size, D), torch.bfloat16)
+    _expect(page_table, "page_table", (N, page_table.shape[1]), torch.int32)
+    _expect(seq_lens, "seq_lens", (N,), torch.int32)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=q.is_pinned())
+    if out.is_cuda or not out.is_contiguous():
+        raise ValueError("out must be a contiguous host tensor")
+    _expect(out, "out", q.shape, torch.bfloat16)
+    dev = torch.cuda.current_device()
+    own = device_buffers is None
+    if own:
+        device_buffers = (torch.empty(q.shape, dtype=torch.bfloat16, device=dev),
+                          torch.empty(k_new.shape, dtype=torch.bfloat16, device=dev),
+                          torch.empty(v_new.shape, dtype=torch.bfloat16, device=dev),
+                          torch.empty(q.shape, dtype=torch.bfloat16, device=dev))
+    qd, kd, vd, od = device_buffers
+    for t, ref, name in ((qd, q, "q_dev"), (kd, k_new, "k_new_dev"), (vd, v_new, "v_new_dev"), (od, q, "out_dev")):
+        _expect(t, name, ref.shape, torch.bfloat16)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    need = attn_decode_paged_workspace_size(N, Hq, D, max_seq_len, page_size)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _need_cuda(qd, kd, vd, od, k_pool, v_pool, page_table, seq_lens, workspace)
+    kernel_stream = torch.cuda.current_stream() if stream is None else stream
+    if kernel_stream != torch.cuda.current_stream():
+        for t in ((qd, kd, vd, od) if own else ()) + ((workspace,) if workspace is not None else ()):
+            t.record_stream(kernel_stream)
+    _release_finished_host_calls()
+    _check("attn_decode_step_host", _lib.load().attn_decode_step_host(
+        _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(out), _ptr(qd), _ptr(kd), _ptr(vd), _ptr(od), _ptr(k_pool),
+        _ptr(v_pool), _ptr(page_table), _ptr(seq_lens), page_size, N, Hq, Hkv, D, num_pages, page_table.shape[1],
+        int(max_seq_len), float(scale), int(window), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+    done = torch.cuda.Event()
+    done.record(kernel_stream)
+    _HOST_IN_FLIGHT.append((done, (q, k_new, v_new, out)))
     return out
 
 

@@ -274,11 +274,11 @@ size_t attn_decode_paged_workspace_size(int N, int Hq, int D, int max_seq_len, i
 
 namespace {
 
-attn_status_t decode_paged(const void* q, const void* k_pool, const void* v_pool, const int32_t* page_table,
-                           const int32_t* seq_lens, int page_size, int N, int Hq, int Hkv, int D, int num_pages,
-                           int max_pages, int max_seq_len, float scale, int window, void* workspace,
-                           size_t workspace_bytes, void* out, attn_stream_t stream, bool fp8, float k_scale,
-                           float v_scale) {
+// Argument checks of the paged decode; ATTN_OK also for an empty batch (N or Hq 0).
+attn_status_t decode_paged_check(const void* q, const void* k_pool, const void* v_pool, const int32_t* page_table,
+                                 const int32_t* seq_lens, int page_size, int N, int Hq, int Hkv, int D, int num_pages,
+                                 int max_pages, int max_seq_len, float scale, int window, const void* workspace,
+                                 size_t workspace_bytes, const void* out, float k_scale, float v_scale) {
   if (N < 0 || Hq < 0 || Hkv < 0 || D <= 0 || num_pages < 0 || max_pages < 0 || max_seq_len < 0 || window < 0 ||
       page_size <= 0)
     return ATTN_ERR_INVALID_ARG;
@@ -298,8 +298,22 @@ attn_status_t decode_paged(const void* q, const void* k_pool, const void* v_pool
   if (G != 1 && G != 2 && G != 4 && G != 8) return ATTN_ERR_UNSUPPORTED;
   if (page_size % 16 != 0 || page_size > 256) return ATTN_ERR_UNSUPPORTED;
   if (N > 65535 || Hkv > 65535) return ATTN_ERR_UNSUPPORTED;
+  // TMA plane coordinates (page * Hkv + g, one page past the pool for boxes outside a sequence) are int32
+  if ((static_cast<long long>(num_pages) + 1) * Hkv > 0x7FFFFFFFLL) return ATTN_ERR_UNSUPPORTED;
   const size_t need = attn::decode_workspace_bytes(N, Hq, D, max_seq_len, page_size);
   if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)) return ATTN_ERR_WORKSPACE;
+  return ATTN_OK;
+}
+
+attn_status_t decode_paged(const void* q, const void* k_pool, const void* v_pool, const int32_t* page_table,
+                           const int32_t* seq_lens, int page_size, int N, int Hq, int Hkv, int D, int num_pages,
+                           int max_pages, int max_seq_len, float scale, int window, void* workspace,
+                           size_t workspace_bytes, void* out, attn_stream_t stream, bool fp8, float k_scale,
+                           float v_scale) {
+  const attn_status_t st = decode_paged_check(q, k_pool, v_pool, page_table, seq_lens, page_size, N, Hq, Hkv, D,
+                                              num_pages, max_pages, max_seq_len, scale, window, workspace,
+                                              workspace_bytes, out, k_scale, v_scale);
+  if (st != ATTN_OK || N == 0 || Hq == 0) return st;
   return from_cuda(attn::launch_decode_paged(q, k_pool, v_pool, page_table, seq_lens, page_size, N, Hq, Hkv, D,
                                              num_pages, max_pages, max_seq_len, scale, window, workspace, out,
                                              attn::device_error_word(), reinterpret_cast<cudaStream_t>(stream), fp8,
@@ -325,6 +339,43 @@ attn_status_t attn_decode_paged_fp8(const void* q, const uint8_t* k_pool, const 
                                     size_t workspace_bytes, void* out, attn_stream_t stream) {
   return decode_paged(q, k_pool, v_pool, page_table, seq_lens, page_size, N, Hq, Hkv, D, num_pages, max_pages,
                       max_seq_len, scale, window, workspace, workspace_bytes, out, stream, true, k_scale, v_scale);
+}
+
+// One serving decode step from and to host memory: copy the step's inputs in,
+// append the new token's K/V, decode, copy the output out, in that order on
+// `stream` (every check happens before anything is enqueued).
+attn_status_t attn_decode_step_host(const void* q_host, const void* k_new_host, const void* v_new_host,
+                                    void* out_host, void* q_dev, void* k_new_dev, void* v_new_dev, void* out_dev,
+                                    void* k_pool, void* v_pool, const int32_t* page_table, const int32_t* seq_lens,
+                                    int page_size, int N, int Hq, int Hkv, int D, int num_pages, int max_pages,
+                                    int max_seq_len, float scale, int window, void* workspace,
+                                    size_t workspace_bytes, attn_stream_t stream) {
+  if (N < 0 || Hq < 0 || Hkv < 0 || D <= 0) return ATTN_ERR_INVALID_ARG;
+  if (N == 0 || Hq == 0) return ATTN_OK;
+  if (q_host == nullptr || k_new_host == nullptr || v_new_host == nullptr || out_host == nullptr ||
+      q_dev == nullptr || k_new_dev == nullptr || v_new_dev == nullptr || out_dev == nullptr)
+    return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(k_new_dev) || !aligned16(v_new_dev)) return ATTN_ERR_INVALID_ARG;
+  // the decode's own checks (the append's are a subset for S_new = 1), before any copy is enqueued
+  attn_status_t st = decode_paged_check(q_dev, k_pool, v_pool, page_table, seq_lens, page_size, N, Hq, Hkv, D,
+                                        num_pages, max_pages, max_seq_len, scale, window, workspace,
+                                        workspace_bytes, out_dev, 1.f, 1.f);
+  if (st != ATTN_OK) return st;
+  if (max_seq_len == 0 || max_pages == 0 || num_pages == 0) return ATTN_ERR_INVALID_ARG;   // nowhere to append
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t q_bytes = static_cast<size_t>(N) * Hq * D * 2, kv_bytes = static_cast<size_t>(N) * Hkv * D * 2;
+  if (cudaMemcpyAsync(q_dev, q_host, q_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(k_new_dev, k_new_host, kv_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(v_new_dev, v_new_host, kv_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  st = attn_kv_append(k_new_dev, v_new_dev, k_pool, v_pool, page_table, seq_lens, page_size, N, Hkv, 1, D,
+                      num_pages, max_pages, stream);
+  if (st != ATTN_OK) return st;
+  st = attn_decode_paged(q_dev, k_pool, v_pool, page_table, seq_lens, page_size, N, Hq, Hkv, D, num_pages,
+                         max_pages, max_seq_len, scale, window, workspace, workspace_bytes, out_dev, stream);
+  if (st != ATTN_OK) return st;
+  return cudaMemcpyAsync(out_host, out_dev, q_bytes, cudaMemcpyDeviceToHost, s) == cudaSuccess ? ATTN_OK
+                                                                                             : ATTN_ERR_CUDA;
 }
 
 attn_status_t attn_decode_paged_noalloc(const void* q, const void* k_pool, const void* v_pool,

@@ -697,10 +697,13 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
   }
 }
 
+}  // namespace
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+namespace {
 EncodeTiledFn g_encoder = nullptr;
 
 void look_up_encoder() {
@@ -717,20 +720,32 @@ EncodeTiledFn tensor_map_encoder() {
   pthread_once(&once, look_up_encoder);
   return g_encoder;
 }
+}  // namespace
+
+bool make_tensor_map_3d(CUtensorMap* m, const void* base, int elem_bytes, int inner, int rows, int planes,
+                        int box_inner, int box_rows) {
+  EncodeTiledFn enc = tensor_map_encoder();
+  if (enc == nullptr || (elem_bytes != 1 && elem_bytes != 2)) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(planes)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner) * elem_bytes,
+                                 static_cast<cuuint64_t>(rows) * inner * elem_bytes};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
+             const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+namespace {
 
 // [planes][rows][D] bf16 tensor, boxes of 64 columns x box_rows rows, 128-byte swizzle.
 bool make_map(CUtensorMap* m, const void* base, int D, int rows, int planes, int box_rows = 128) {
-  EncodeTiledFn enc = tensor_map_encoder();
-  if (enc == nullptr) return false;
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
-                              static_cast<cuuint64_t>(planes)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(rows) * D * 2};
-  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return make_tensor_map_3d(m, base, 2, D, rows, planes, 64, box_rows);
 }
+
+}  // namespace
 
 int sm_count() {
   constexpr int kMaxDevices = 64;
@@ -744,6 +759,8 @@ int sm_count() {
   }
   return cache[dev];
 }
+
+namespace {
 
 // One-time set-up of a kernel on the current device: its shared-memory limit,
 // and the check that setmaxnreg.inc can be honoured (it waits until the

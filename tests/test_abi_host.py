@@ -251,3 +251,20 @@ def test_host_prefill_argument_validation():
     assert call(chunks=5) == 1                   # more pieces than (batch, kv head) pairs (2 x 2)
     assert call(D=96) == 1
     assert call(B=0, qh=None, oh=None, qd=None, od=None) == 0   # empty problem
+
+
+def test_host_decode_step_argument_validation():
+    lib = _lib()
+
+    def call(qh=FAKE, kh=FAKE, oh=FAKE, qd=FAKE, kd=FAKE, N=4, Hq=8, Hkv=2, D=128, page=16, ws=FAKE, msl=256):
+        return lib.attn_decode_step_host(qh, kh, FAKE, oh, qd, kd, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, page, N, Hq,
+                                         Hkv, D, 64, 16, msl, 0.1, 0, ws, 1 << 30, None)
+    assert call(qh=None) == 1                    # host buffers are required
+    assert call(oh=None) == 1
+    assert call(kd=None) == 1                    # and the device ones
+    assert call(kd=MISALIGNED) == 1
+    assert call(D=96) == 1
+    assert call(Hq=24, Hkv=2) == 2               # group of 12
+    assert call(ws=None) == 6
+    assert call(msl=0) == 1                      # no room to append the new token
+    assert call(N=0, qh=None, oh=None) == 0      # empty batch
