@@ -50,6 +50,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "common.cuh"
 #include "sm100_ptx.cuh"
@@ -68,7 +69,7 @@ constexpr int kBox = 16;          // rows per page box (every supported page siz
 constexpr int kSWarp = 4;
 constexpr int kPvWarp = 5;
 constexpr int kLoadWarp0 = 6;
-constexpr int kThreads = 320;
+constexpr int kConvWarp0 = 10;    // 8-bit caches: warps 10-13 rewrite the codes as f16 in place
 constexpr float kTau = 8.0f;      // lazy-rescale threshold, log2 units
 
 template <int D>
@@ -86,12 +87,16 @@ struct TcCfg {
   static constexpr uint32_t O_COL = 0;
   static constexpr uint32_t S_COL = 2 * D;
   static constexpr uint32_t TMEM_COLS = (S_COL + 2 * kNH <= 256) ? 256 : 512;
-  static constexpr int TAIL = 1280;                     // barriers and reduction scratch
+  static constexpr int BAR_BYTES = 512;                 // mbarriers, the TMEM address and the abort flag
+  static constexpr int TAIL = BAR_BYTES + 1024;         // + reduction scratch
   static constexpr size_t SMEM = 1024 + 2 * Q_BYTES + 2 * P_BYTES + kSlots * TILE_BYTES + TAIL;
 };
 
+template <bool FP8>
+constexpr int tc_threads() { return FP8 ? 448 : 320; }
+
 struct TcParams {
-  const void* k_pool;   // [num_pages, Hkv, page_size, D] bf16
+  const void* k_pool;   // [num_pages, Hkv, page_size, D] bf16, or E4M3 codes
   const void* v_pool;
   const int32_t* page_table;
   const int32_t* seq_lens;
@@ -132,11 +137,18 @@ __device__ __forceinline__ DItem item_at(const TcParams& p, int k, int len) {
   return it;
 }
 
-template <int D, int G>
-__global__ void __launch_bounds__(kThreads, 1)
+// FP8: the pools hold E4M3 codes.  Their tiles arrive row-major in the upper
+// half of a slot (one box of 16 rows x D bytes per page of one head); converter
+// warps rewrite each in place as f16 (exact for every code) in the layout the
+// MMA reads, and the queries and P are f16 as well, so the products run on f16
+// operands.  The K scale is folded into the softmax scale, the V scale into the
+// combine.
+template <int D, int G, bool FP8>
+__global__ void __launch_bounds__(tc_threads<FP8>(), 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v, const TcParams p) {
   using C = TcCfg<D>;
+  constexpr int RAW_OFF = C::TILE_BYTES / 2;            // FP8: where a slot's codes land (row-major)
   static_assert(G >= 1 && G <= kNH, "group size");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -156,9 +168,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* o_full = p_free + 2;                        // 2: an item's last product into O buffer done
   uint64_t* o_free = o_full + 2;                        // 2: O buffer read out
   uint64_t* drain = o_free + 2;                         // 2: each issuer's products complete
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
+  uint64_t* raw_full = drain + 2;                       // kSlots (FP8): a slot's codes have landed
+  uint64_t* q_conv = raw_full + kSlots;                 // 2 (FP8): queries rewritten as f16
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_conv + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* red = reinterpret_cast<float*>(tail + 256);    // [2][4 warps][16]: tile maxima
+  static_assert((2 + 2 + kSlots + kSlots + 6 * 2 + 2 + kSlots + 2) * 8 + 8 <= C::BAR_BYTES, "barrier area");
+  float* red = reinterpret_cast<float*>(tail + C::BAR_BYTES);   // [2][4 warps][16]: tile maxima
   float* lred = red + 2 * 4 * kNH;                      // [4 warps][16]: row sums
   volatile int* okv = reinterpret_cast<volatile int*>(lred + 4 * kNH);   // [3][4 warps]: status at a barrier
 
@@ -177,9 +192,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&o_free[i], 128);
     }
     for (int s = 0; s < kSlots; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], FP8 ? 32 : 1);   // FP8: the converter warp's lanes; bf16: the TMA bytes
       mbar_init(&empty[s], 1);
+      mbar_init(&raw_full[s], 1);
     }
+    mbar_init(&q_conv[0], 32);
+    mbar_init(&q_conv[1], 32);
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
     *abort_flag = 0;
@@ -200,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp >= kLoadWarp0) {
+  if (warp >= kLoadWarp0 && warp < kConvWarp0) {
     // ------------------------------------------------------------ loader warps 6-9
     // K tiles go to a ring of kKSlots slots, V tiles to a ring of kVSlots:
     // each ring has one consumer (the S^T issuer, the P V issuer) that takes
@@ -270,9 +288,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         int ph = __shfl_sync(0xffffffffu, ph_it, (jj * 8 + rb) & 31);
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(&empty[st], ((t / nslots) & 1) ^ 1, abort_flag, p.err))))
           break;
-        if (lane == 0) mbar_arrive_expect_tx(&full[st], C::TILE_BYTES);
+        uint64_t* bar = FP8 ? &raw_full[st] : &full[st];
+        if (lane == 0) mbar_arrive_expect_tx(bar, FP8 ? kBT * D : C::TILE_BYTES);
         __syncwarp();   // the barrier is armed before any box can land
-        if (lane < 8 * C::KATOMS) {
+        if (lane < (FP8 ? 8 : 8 * C::KATOMS)) {
           const int tok0 = (it.j0 + jj) * kBT + rb * kBox;
           if (!(tok0 + kBox > it.t_begin && tok0 < it.t_end)) {
             ph = p.num_pages;   // no key of the item: a plane past the pool, read as zeros
@@ -280,17 +299,107 @@ __global__ void __launch_bounds__(kThreads, 1)
             record_error(p.err, ATTN_ERRBIT_BADPAGE);
             ph = 0;
           }
-          tma_load_3d(sRing + st * C::TILE_BYTES + a * C::ATOM_BYTES + rb * kBox * 128,
-                      load_v ? &tmap_v : &tmap_k, &full[st], a * 64, tok0 % p.page_size, ph * p.Hkv + it.g);
+          if constexpr (FP8)   // one box per page of the head: 16 rows x D codes, row-major
+            tma_load_3d(sRing + st * C::TILE_BYTES + RAW_OFF + rb * kBox * D, load_v ? &tmap_v : &tmap_k, bar, 0,
+                        tok0 % p.page_size, ph * p.Hkv + it.g);
+          else
+            tma_load_3d(sRing + st * C::TILE_BYTES + a * C::ATOM_BYTES + rb * kBox * 128,
+                        load_v ? &tmap_v : &tmap_k, bar, a * 64, tok0 % p.page_size, ph * p.Hkv + it.g);
         }
       }
       T += it.nt;
     }
     // this warp's last copies must land before the CTA may exit (normally consumed already)
     for (int t = T - 1; t >= 0 && t >= T - nslots; --t)
-      if ((t % nslots) % 2 == wl) mbar_wait(&full[slot0 + t % nslots], (t / nslots) & 1, nullptr, p.err);
+      if ((t % nslots) % 2 == wl)
+        mbar_wait(FP8 ? &raw_full[slot0 + t % nslots] : &full[slot0 + t % nslots], (t / nslots) & 1, nullptr,
+                  p.err);
     if (lw == 0 && lane == 0)
       for (int m = max(0, qn - 2); m < qn; ++m) mbar_wait(&q_full[m & 1], (m >> 1) & 1, nullptr, p.err);
+  } else if (FP8 && warp >= kConvWarp0) {
+    // ------------------------------------------------------------ converter warps 10-13 (FP8)
+    // Warps 10, 11 rewrite the K tiles t with t % kKSlots % 2 = 0, 1, warps 12,
+    // 13 the V tiles likewise: each slot has one converter, which takes that
+    // slot's tiles in order.  A slot's D-byte rows of codes sit row-major in its
+    // upper half; the converter turns them into f16 in the 128-byte-swizzled
+    // layout of a 16-bit tile, in place.  Rows go in increasing order, 32 or 64
+    // at a time, each batch read completely before any of it is written: the
+    // f16 row r lands on code rows of its own batch or earlier ones, never on a
+    // code row still to be read.  Warp 10 also rewrites each
+    // item's queries (bf16, landed by TMA) as f16 in place.
+    const int cw = warp - kConvWarp0;
+    const bool conv_v = cw >= 2;
+    const int nslots = conv_v ? kVSlots : kKSlots;
+    const int slot0 = conv_v ? kKSlots : 0;
+    const int wl = cw & 1;
+    constexpr int LPR = D / 16;                       // lanes per row: 16 codes (one 16-byte load) each
+    constexpr int RPS = 32 / LPR;                     // rows per step
+    const int lr = lane / LPR, c = lane % LPR;        // row within the step, 16-code chunk of the row
+    int T = 0, qn = 0;
+    bool ok = true;
+    int len_cur = item_len(p, blockIdx.x);
+    for (int r = 0; r < n_rounds && ok; ++r) {
+      const int k = blockIdx.x + r * gridDim.x;
+      const int len_next = item_len(p, k + gridDim.x);
+      const DItem it = item_at(p, k, len_cur);
+      len_cur = len_next;
+      if (it.nt == 0) continue;
+      if (cw == 0) {   // the item's queries: bf16 -> f16, in place
+        const int qb = qn & 1;
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&q_full[qb], (qn >> 1) & 1, abort_flag, p.err)))) break;
+        uint4* qv = reinterpret_cast<uint4*>(sQ + qb * C::Q_BYTES);
+        for (int i = lane; i < C::Q_BYTES / 16; i += 32) {   // every row (rows past q_rows feed ignored columns)
+          uint4 u = qv[i];
+          uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __half2 h = __floats2half2_rn(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u));
+            w[e] = *reinterpret_cast<const uint32_t*>(&h);
+          }
+          qv[i] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&q_conv[qb]);
+      }
+      ++qn;
+      for (int jj = 0; jj < it.nt && ok; ++jj) {
+        const int t = T + jj;
+        const int rs = t % nslots;
+        if (rs % 2 != wl) continue;
+        const int st = slot0 + rs;
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&raw_full[st], (t / nslots) & 1, abort_flag, p.err)))) break;
+        uint8_t* slot = sRing + st * C::TILE_BYTES;
+        const uint4* raw = reinterpret_cast<const uint4*>(slot + RAW_OFF);
+        constexpr int BATCH = 8;                      // steps whose codes are read before any is written
+        for (int r0 = 0; r0 < kBT; r0 += RPS * BATCH) {
+          uint4 u[BATCH];
+#pragma unroll
+          for (int b = 0; b < BATCH; ++b) u[b] = raw[(r0 + b * RPS + lr) * LPR + c];
+          __syncwarp();   // the batch's code rows are read before any of its f16 rows is written
+#pragma unroll
+          for (int b = 0; b < BATCH; ++b) {
+            const int row = r0 + b * RPS + lr;
+            const uint32_t w[4] = {u[b].x, u[b].y, u[b].z, u[b].w};
+            uint32_t h[8];   // 16 f16: elements 16 c .. 16 c + 15 of the row
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const unsigned short lo = static_cast<unsigned short>(w[e]), hi = static_cast<unsigned short>(w[e] >> 16);
+              asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h[2 * e]) : "h"(lo));
+              asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h[2 * e + 1]) : "h"(hi));
+            }
+            // two 16-byte chunks of atom (16 c) / 64, chunks 2 (c % 4) and 2 (c % 4) + 1 of the row, swizzled
+            const int atom = c / 4, q0 = 2 * (c % 4);
+            uint8_t* rowp = slot + atom * C::ATOM_BYTES + row * 128;
+            *reinterpret_cast<uint4*>(rowp + ((q0 ^ (row & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
+            *reinterpret_cast<uint4*>(rowp + (((q0 + 1) ^ (row & 7)) << 4)) = make_uint4(h[4], h[5], h[6], h[7]);
+          }
+          __syncwarp();
+        }
+        fence_proxy_async_smem();   // the tensor cores read the tile through the async proxy
+        mbar_arrive(&full[st]);
+      }
+      T += it.nt;
+    }
   } else if (warp == kSWarp || warp == kPvWarp) {
     // ------------------------------------------------------------ MMA issuers
     // Two threads issue the products, so that the issue cost of one (tens of
@@ -299,8 +408,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Tile t's K is load t of the K ring and its V load t of the V ring.
     if (lane == 0) {
       const bool is_s = (warp == kSWarp);
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, kNH, 0, 0);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(64, D, 0, 1);
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, kNH, 0, 0, FP8);   // FP8: f16 operands
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(64, D, 0, 1, FP8);
       constexpr uint32_t kHi = sw128_desc_hi(1024);   // 8-row groups 1024 B apart
       const uint32_t q_lo0 = sw128_desc_lo(smem_u32(sQ), 16);
       const uint32_t p_lo0 = sw128_desc_lo(smem_u32(sP), 16);
@@ -349,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (it.nt == 0) continue;
         if (is_s) {
           const int qb = qn & 1;
-          if (!(ok = mbar_wait(&q_full[qb], (qn >> 1) & 1, abort_flag, p.err))) break;
+          if (!(ok = mbar_wait(FP8 ? &q_conv[qb] : &q_full[qb], (qn >> 1) & 1, abort_flag, p.err))) break;
           tc_fence_after();
           for (int jj = 0; jj < it.nt && ok; ++jj) {
             const int t = T + jj, sb = t & 1;
@@ -508,10 +617,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int chunk = (rl & 63) >> 3;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          const __nv_bfloat16 v = __float2bfloat16_rn(pr[h]);
+          unsigned short v;
+          if constexpr (FP8) {
+            const __half hv = __float2half_rn(pr[h]);
+            v = *reinterpret_cast<const unsigned short*>(&hv);
+          } else {
+            const __nv_bfloat16 bv = __float2bfloat16_rn(pr[h]);
+            v = *reinterpret_cast<const unsigned short*>(&bv);
+          }
           const uint32_t addr = pbase + h * 128 + ((chunk ^ (h & 7)) << 4);
-          asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(*reinterpret_cast<const unsigned short*>(&v))
-                       : "memory");
+          asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
         }
         fence_proxy_async_smem();   // the MMA reads P through the async proxy
         tc_fence_before();
@@ -574,11 +689,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, int G>
+template <int D, int G, bool FP8>
 cudaError_t launch_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const TcParams& p,
                      cudaStream_t stream) {
   using C = TcCfg<D>;
-  auto kern = decode_tc_kernel<D, G>;
+  auto kern = decode_tc_kernel<D, G, FP8>;
   constexpr int kMaxDevices = 64;
   static int ready[kMaxDevices] = {};   // the shared-memory limit is set once per device
   int dev = 0;
@@ -592,7 +707,7 @@ cudaError_t launch_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   const int sms = sm_count();
   if (sms <= 0) return cudaErrorInvalidDevice;
   const unsigned grid = static_cast<unsigned>(p.n_items < sms ? p.n_items : sms);
-  kern<<<grid, kThreads, C::SMEM, stream>>>(mq, mk, mv, p);
+  kern<<<grid, tc_threads<FP8>(), C::SMEM, stream>>>(mq, mk, mv, p);
   return cudaGetLastError();
 }
 
@@ -602,7 +717,7 @@ cudaError_t launch_decode_tc_split(const void* q, const void* k_pool, const void
                                    const int32_t* seq_lens, int page_size, int N, int Hq, int Hkv, int D,
                                    int num_pages, int max_pages, int max_seq_len, float scale, int window,
                                    int split_tokens, int max_splits, float* ws_o, float* ws_lse, unsigned int* err,
-                                   cudaStream_t stream) {
+                                   cudaStream_t stream, bool fp8, float k_scale) {
   const int G = Hq / Hkv;
   if (split_tokens % kBT != 0 || page_size % kBox != 0) return cudaErrorInvalidValue;
   TcParams p{};
@@ -627,15 +742,18 @@ cudaError_t launch_decode_tc_split(const void* q, const void* k_pool, const void
   if (items > (1LL << 30)) return cudaErrorInvalidValue;
   p.n_items = static_cast<int>(items);
   p.q_rows = Hq < kNH ? Hq : kNH;
-  p.scale_log2 = scale * 1.4426950408889634f;
+  p.scale_log2 = scale * k_scale * 1.4426950408889634f;
   CUtensorMap mq, mk, mv;
+  // bf16 pools: 64-column boxes in the 128-byte swizzle; 8-bit pools: whole D-byte rows, row-major
+  const int eb = fp8 ? 1 : 2, box_inner = fp8 ? D : 64;
   if (!make_tensor_map_3d(&mq, q, 2, D, Hq, N, 64, p.q_rows) ||
-      !make_tensor_map_3d(&mk, k_pool, 2, D, page_size, num_pages * Hkv, 64, kBox) ||
-      !make_tensor_map_3d(&mv, v_pool, 2, D, page_size, num_pages * Hkv, 64, kBox))
+      !make_tensor_map_3d(&mk, k_pool, eb, D, page_size, num_pages * Hkv, box_inner, kBox, !fp8) ||
+      !make_tensor_map_3d(&mv, v_pool, eb, D, page_size, num_pages * Hkv, box_inner, kBox, !fp8))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaErrorInvalidValue;
-#define ATTN_TC_CASE(DD, GG) \
-  if (D == DD && G == GG) e = launch_d<DD, GG>(mq, mk, mv, p, stream);
+#define ATTN_TC_CASE(DD, GG)                                                              \
+  if (D == DD && G == GG)                                                                 \
+    e = fp8 ? launch_d<DD, GG, true>(mq, mk, mv, p, stream) : launch_d<DD, GG, false>(mq, mk, mv, p, stream);
   ATTN_TC_CASE(128, 1) ATTN_TC_CASE(128, 2) ATTN_TC_CASE(128, 4) ATTN_TC_CASE(128, 8)
   ATTN_TC_CASE(64, 1) ATTN_TC_CASE(64, 2) ATTN_TC_CASE(64, 4) ATTN_TC_CASE(64, 8)
 #undef ATTN_TC_CASE

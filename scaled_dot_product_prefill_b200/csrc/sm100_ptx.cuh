@@ -264,12 +264,12 @@ __device__ __forceinline__ uint64_t desc64(uint32_t lo, uint32_t hi) {
   return d;
 }
 
-// Instruction descriptor, kind::f16 with bf16 A and B and an fp32 accumulator.
-// a_mn / b_mn select MN-major operands (1) instead of K-major (0).
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn) {
+// Instruction descriptor, kind::f16 with bf16 (or, with f16 = true, f16) A and B and
+// an fp32 accumulator.  a_mn / b_mn select MN-major operands (1) instead of K-major (0).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn, bool f16 = false) {
   return (1u << 4)                                   // D format: f32
-         | (1u << 7)                                 // A format: bf16
-         | (1u << 10)                                // B format: bf16
+         | (f16 ? 0u : (1u << 7))                    // A format: bf16 (1) or f16 (0)
+         | (f16 ? 0u : (1u << 10))                   // B format: bf16 (1) or f16 (0)
          | (static_cast<uint32_t>(a_mn) << 15)       // A major
          | (static_cast<uint32_t>(b_mn) << 16)       // B major
          | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
