@@ -22,8 +22,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libattn_b200.so")
 
-SOURCES = ["attn_api.cu", "prefill_sm100.cu", "prefill_f32.cu", "decode_paged.cu", "decode_tc.cu", "kv_append.cu",
-           "page_pool.cpp"]
+SOURCES = ["attn_api.cu", "prefill_sm100.cu", "prefill_f32.cu", "decode_paged.cu", "kv_append.cu", "page_pool.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 # Host code is built without exceptions and uses only the C library and
 # pthreads, so the .so needs no C++ runtime: a late dlopen of libstdc++ can

@@ -298,8 +298,6 @@ attn_status_t decode_paged_check(const void* q, const void* k_pool, const void* 
   if (G != 1 && G != 2 && G != 4 && G != 8) return ATTN_ERR_UNSUPPORTED;
   if (page_size % 16 != 0 || page_size > 256) return ATTN_ERR_UNSUPPORTED;
   if (N > 65535 || Hkv > 65535) return ATTN_ERR_UNSUPPORTED;
-  // TMA plane coordinates (page * Hkv + g, one page past the pool for boxes outside a sequence) are int32
-  if ((static_cast<long long>(num_pages) + 1) * Hkv > 0x7FFFFFFFLL) return ATTN_ERR_UNSUPPORTED;
   const size_t need = attn::decode_workspace_bytes(N, Hq, D, max_seq_len, page_size);
   if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)) return ATTN_ERR_WORKSPACE;
   return ATTN_OK;

@@ -26,10 +26,10 @@ __device__ __forceinline__ void record_error(unsigned int* err, unsigned int bit
 unsigned int* device_error_word();
 
 // 3-D tensor map over [planes][rows][inner] elements of elem_bytes bytes (2: bf16, 1: bytes),
-// boxes of box_inner x box_rows x 1, with the 128-byte swizzle or none (a box then lands
-// row-major).  False if the driver's encoder is unavailable or rejects the map.
+// boxes of box_inner x box_rows x 1, 128-byte swizzle.  False if the driver's encoder is
+// unavailable or rejects the map.
 bool make_tensor_map_3d(CUtensorMap* m, const void* base, int elem_bytes, int inner, int rows, int planes,
-                        int box_inner, int box_rows, bool swizzle = true);
+                        int box_inner, int box_rows);
 
 // Number of SMs of the current device (cached per device), 0 on error.
 int sm_count();
@@ -63,16 +63,6 @@ cudaError_t launch_decode_paged(const void* q, const void* k_pool, const void* v
                                 int num_pages, int max_pages, int max_seq_len, float scale, int window,
                                 void* workspace, void* out, unsigned int* err, cudaStream_t stream,
                                 bool fp8 = false, float k_scale = 1.f, float v_scale = 1.f);
-
-// The split pass of the paged decode on the tensor cores (bf16 cache, or E4M3 codes with fp8):
-// normalised partial outputs ws_o
-// [N, Hq, max_splits, D] and base-2 log-sum-exps ws_lse [N, Hq, max_splits] of every split that
-// holds a visible key (split_tokens a multiple of 128; page_size a multiple of 16).
-cudaError_t launch_decode_tc_split(const void* q, const void* k_pool, const void* v_pool, const int32_t* page_table,
-                                   const int32_t* seq_lens, int page_size, int N, int Hq, int Hkv, int D,
-                                   int num_pages, int max_pages, int max_seq_len, float scale, int window,
-                                   int split_tokens, int max_splits, float* ws_o, float* ws_lse, unsigned int* err,
-                                   cudaStream_t stream, bool fp8 = false, float k_scale = 1.f);
 
 // k_new/v_new [B, Hkv, S_new, D] -> pools [num_pages, Hkv, page_size, D] at positions seq_lens[b] - S_new + i.
 cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* k_pool, void* v_pool,

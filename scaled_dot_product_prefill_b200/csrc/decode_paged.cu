@@ -512,7 +512,7 @@ DecodeGeometry decode_geometry(int N, int Hq, int D, int max_seq_len, int page_s
   // to fill the GPU.
   int split = kSplit;
   const long long units = static_cast<long long>(N);
-  while (split > 128 && units * ((max_seq_len + split - 1) / split) < 1024) split /= 2;
+  while (split > 64 && units * ((max_seq_len + split - 1) / split) < 1024) split /= 2;
   g.split_tokens = split;
   g.max_splits = max_seq_len > 0 ? (max_seq_len + split - 1) / split : 1;
   return g;
@@ -556,13 +556,9 @@ cudaError_t launch_decode_paged(const void* q, const void* k_pool, const void* v
   p.out = static_cast<__nv_bfloat16*>(out);
   const int G = Hq / Hkv;
   cudaError_t e = cudaErrorInvalidValue;
-  if (fp8) {   // 8-bit cache: both contractions on the tensor cores (decode_tc.cu)
-    e = launch_decode_tc_split(q, k_pool, v_pool, page_table, seq_lens, page_size, N, Hq, Hkv, D, num_pages,
-                               max_pages, max_seq_len, scale, window, geo.split_tokens, geo.max_splits, p.ws_o,
-                               p.ws_lse, err, stream, true, k_scale);
-  }
-#define ATTN_DECODE_CASE(DD, GG) \
-  if (!fp8 && D == DD && G == GG) e = launch_split<DD, GG, false>(p, N, stream);
+#define ATTN_DECODE_CASE(DD, GG)                                        \
+  if (D == DD && G == GG)                                               \
+    e = fp8 ? launch_split<DD, GG, true>(p, N, stream) : launch_split<DD, GG, false>(p, N, stream);
   ATTN_DECODE_CASE(128, 1) ATTN_DECODE_CASE(128, 2) ATTN_DECODE_CASE(128, 4) ATTN_DECODE_CASE(128, 8)
   ATTN_DECODE_CASE(64, 1) ATTN_DECODE_CASE(64, 2) ATTN_DECODE_CASE(64, 4) ATTN_DECODE_CASE(64, 8)
 #undef ATTN_DECODE_CASE

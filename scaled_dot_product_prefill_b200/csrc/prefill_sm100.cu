@@ -723,7 +723,7 @@ EncodeTiledFn tensor_map_encoder() {
 }  // namespace
 
 bool make_tensor_map_3d(CUtensorMap* m, const void* base, int elem_bytes, int inner, int rows, int planes,
-                        int box_inner, int box_rows, bool swizzle) {
+                        int box_inner, int box_rows) {
   EncodeTiledFn enc = tensor_map_encoder();
   if (enc == nullptr || (elem_bytes != 1 && elem_bytes != 2)) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows),
@@ -734,7 +734,7 @@ bool make_tensor_map_3d(CUtensorMap* m, const void* base, int elem_bytes, int in
   const cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 

@@ -204,18 +204,6 @@ __device__ __forceinline__ void tmem_ld32f(uint32_t taddr, float* r) {
       : "memory");
 }
 
-// 32 lanes x 16 consecutive 32-bit columns, as floats.
-__device__ __forceinline__ void tmem_ld16f(uint32_t taddr, float* r) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=f"(r[0]), "=f"(r[1]), "=f"(r[2]), "=f"(r[3]), "=f"(r[4]), "=f"(r[5]), "=f"(r[6]), "=f"(r[7]),
-        "=f"(r[8]), "=f"(r[9]), "=f"(r[10]), "=f"(r[11]), "=f"(r[12]), "=f"(r[13]), "=f"(r[14]),
-        "=f"(r[15])
-      : "r"(taddr)
-      : "memory");
-}
-
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -226,11 +214,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
       "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
       "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
-}
-
-// Named barrier `id` (1..15) over `count` threads (a multiple of 32); id 0 is __syncthreads.
-__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // ----------------------------------------------------------------- descriptors
@@ -264,12 +247,12 @@ __device__ __forceinline__ uint64_t desc64(uint32_t lo, uint32_t hi) {
   return d;
 }
 
-// Instruction descriptor, kind::f16 with bf16 (or, with f16 = true, f16) A and B and
-// an fp32 accumulator.  a_mn / b_mn select MN-major operands (1) instead of K-major (0).
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn, bool f16 = false) {
+// Instruction descriptor, kind::f16 with bf16 A and B and an fp32 accumulator.
+// a_mn / b_mn select MN-major operands (1) instead of K-major (0).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn) {
   return (1u << 4)                                   // D format: f32
-         | (f16 ? 0u : (1u << 7))                    // A format: bf16 (1) or f16 (0)
-         | (f16 ? 0u : (1u << 10))                   // B format: bf16 (1) or f16 (0)
+         | (1u << 7)                                 // A format: bf16
+         | (1u << 10)                                // B format: bf16
          | (static_cast<uint32_t>(a_mn) << 15)       // A major
          | (static_cast<uint32_t>(b_mn) << 16)       // B major
          | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8

@@ -48,12 +48,9 @@ def test_fp8_decode_matches_oracle(case):
     assert_parity(out, ref, "bf16", str(case))
 
 
-def test_fp8_decode_agrees_with_the_bf16_decode_of_the_decoded_cache():
-    """With power-of-two scales every decoded element is exact in bf16, so the bf16 decode of the decoded cache
-    sees the same numbers as the 8-bit decode: both match the oracle, and each other within the bf16 tolerance.
-
-    (The two caches run different kernels: the 8-bit one on CUDA cores, the bf16 one on the tensor cores with
-    P rounded to bf16, so their outputs need not agree bit for bit.)"""
+def test_fp8_decode_equals_bf16_decode_of_the_decoded_cache():
+    """With power-of-two scales every decoded element is exact in bf16 and every scaling is exact in fp32:
+    the 8-bit path must then return the bf16 path's output bit for bit, and both match the oracle."""
     ks, vs = 1 / 64, 1 / 128
     p = inputs.paged_inputs_fp8(6, 32, 8, 128, 16, seed=5, k_scale=ks, v_scale=vs,
                                 seq_lens=[33, 1000, 17, 4097, 250, 64])
@@ -65,10 +62,8 @@ def test_fp8_decode_agrees_with_the_bf16_decode_of_the_decoded_cache():
     out16 = api.attn_decode_paged(*dev, max_seq_len=p.max_seq_len)
     torch.cuda.synchronize()
     assert api.attn_device_status(clear=True) == 0
-    ref = oracle_fp8(p, ks, vs, 1 / np.sqrt(128), 0)
-    assert_parity(out8, ref, "bf16", "8-bit cache")
-    assert_parity(out16, ref, "bf16", "bf16 decode of the decoded cache")
-    assert (out8.float() - out16.float()).abs().max().item() <= 2e-2
+    assert torch.equal(out8, out16)
+    assert_parity(out8, oracle_fp8(p, ks, vs, 1 / np.sqrt(128), 0), "bf16", "8-bit cache")
 
 
 def test_fp8_decode_workload_every_sequence():
