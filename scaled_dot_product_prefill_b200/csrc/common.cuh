@@ -25,6 +25,35 @@ __device__ __forceinline__ void record_error(unsigned int* err, unsigned int bit
 // Device address of this device's error word (looked up once per device).
 unsigned int* device_error_word();
 
+// Programmatic dependent launch.  A kernel launched with launch_dependent()
+// may be scheduled before the kernel ahead of it in the stream has finished,
+// so that its launch and set-up overlap that kernel's tail.  Every such kernel
+// calls grid_dependency_wait() before its first access to global memory: the
+// wait returns once the preceding grid has completed and its writes are
+// visible (at once when there is no such grid).  grid_dependents_may_start()
+// lets the next kernel be scheduled before this one ends; it does not make
+// this kernel's writes visible early.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependents_may_start() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... Params, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                             Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Params>(args)...);
+}
+
 // 3-D tensor map over [planes][rows][inner] elements of elem_bytes bytes (2: bf16, 1: bytes),
 // boxes of box_inner x box_rows x 1, 128-byte swizzle.  False if the driver's encoder is
 // unavailable or rejects the map.

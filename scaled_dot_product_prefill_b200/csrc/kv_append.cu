@@ -64,6 +64,8 @@ __global__ void __launch_bounds__(kThreads) kv_append_kernel(const uint4* __rest
                                                              int B, int Hkv, int S_new, int pieces, int num_pages,
                                                              int max_pages, unsigned int* err, float k_inv,
                                                              float v_inv) {
+  grid_dependency_wait();   // the pools may still be read by the kernel before
+  grid_dependents_may_start();
   const unsigned int total = static_cast<unsigned int>(B) * Hkv * S_new * pieces;
   const unsigned int pass = gridDim.x * kThreads * kUnroll;
   for (unsigned int base = blockIdx.x * kThreads * kUnroll + threadIdx.x; base < total; base += pass) {
@@ -133,10 +135,9 @@ cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* k_pool,
   const long long want = (total + kThreads * kUnroll - 1) / (kThreads * kUnroll);
   const int grid = static_cast<int>(want < 8LL * n_sm ? want : 8LL * n_sm);
   auto kern = fp8 ? kv_append_kernel<true> : kv_append_kernel<false>;
-  kern<<<grid, kThreads, 0, stream>>>(static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), k_pool,
-                                      v_pool, page_table, seq_lens, page_size, B, Hkv, S_new, pieces, num_pages,
-                                      max_pages, err, 1.f / k_scale, 1.f / v_scale);
-  return cudaGetLastError();
+  return launch_dependent(kern, dim3(grid), dim3(kThreads), 0, stream, static_cast<const uint4*>(k_new),
+                          static_cast<const uint4*>(v_new), k_pool, v_pool, page_table, seq_lens, page_size, B, Hkv,
+                          S_new, pieces, num_pages, max_pages, err, 1.f / k_scale, 1.f / v_scale);
 }
 
 }  // namespace attn

@@ -238,6 +238,8 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // set-up above overlaps the tail of the kernel before; global memory only from here on
+  grid_dependency_wait();
 
   if (warp >= 8) {
    // ------------------------------------------------------------ producer warpgroup
@@ -798,8 +800,7 @@ cudaError_t launch_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   const int sms = sm_count();
   if (sms <= 0) return cudaErrorInvalidDevice;
   const unsigned grid = static_cast<unsigned>(min(p.n_items, sms));
-  kern<<<grid, C::THREADS, smem, stream>>>(mq, mk, mv, p);
-  return cudaGetLastError();
+  return launch_dependent(kern, dim3(grid), dim3(C::THREADS), smem, stream, mq, mk, mv, p);
 }
 
 }  // namespace

@@ -114,7 +114,7 @@ def test_sequence_longer_than_hint_is_reported():
 
 
 def test_long_context_decode_merges_more_than_32_splits():
-    """70k tokens at 512 keys per split: the combine walks its splits in several blocks of 32."""
+    """Two sequences of up to 70k tokens take 274 splits of 256 keys: the combine walks them in blocks of 32."""
     p = inputs.paged_inputs(2, 8, 2, 128, 16, seed=77, seq_lens=[40000, 70001], spare_pages=4, poison=True)
     out = run_decode(p)
     assert api.attn_device_status(clear=True) == 0
