@@ -167,9 +167,11 @@ attn_status_t attn_prefill_lse(const void* q, const void* k, const void* v, void
  * q_dev, k_dev, v_dev, out_dev : device buffers of the same sizes, owned by
  *     the caller (the library allocates nothing), 16-byte aligned; their
  *     contents are overwritten.  k/v buffers may be null when Skv == 0.
- * chunks : pieces, 1 .. B * Hkv; 0 = two (one if B * Hkv == 1).  The
- *     host link bounds the call and each piece adds some copy and launch
- *     latency, so a few pieces do best.
+ * chunks : pieces, 1 .. B * Hkv; 0 = one piece per 48 MB of input,
+ *     rounded, at least two and at most eight (at most B * Hkv).  The host
+ *     link bounds the call; more pieces shorten the last piece's kernel and
+ *     copy back, which follow the last input copy, and each piece adds some
+ *     copy and launch latency.
  * stream : the stream of the kernels.  When `stream` completes, every copy
  *     of the call has completed; the copies start only after work that was
  *     on `stream` before the call.

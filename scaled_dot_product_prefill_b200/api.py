@@ -128,7 +128,7 @@ def attn_prefill_host(q, k, v, *, causal=False, window=0, scale=None, out=None, 
     """bf16 prefill whose q [B,Hq,Sq,D], k/v [B,Hkv,Skv,D] and output are host (CPU) tensors.
 
     The C call copies the inputs to the device, runs the prefill and copies
-    the output back, in `chunks` pieces (0: two) so that the copies overlap
+    the output back, in `chunks` pieces (0: one per 48 MB of input, 2 to 8) so that the copies overlap
     the kernels; page-locked host tensors (``pin_memory()``) are needed for
     the overlap.  `device_buffers` = (q_dev, k_dev, v_dev, out_dev) CUDA
     tensors of the same shapes, allocated here if None.  `copy_streams` =
