@@ -27,6 +27,7 @@ SMALL = [
     (5, 32, 8, 128, 16, [4096, 1, 511, 512, 2500], 0),
     (4, 8, 2, 128, 16, [300, 1200, 20, 4000], 100),   # sliding window over the cache
     (2, 8, 4, 64, 16, [1, 0], 0),                # an empty cache gives zeros
+    (3, 16, 4, 64, 16, [2100, 47, 900], 0),      # group of 4 at D = 64 (two score pieces per lane)
 ]
 
 
@@ -111,6 +112,17 @@ def test_sequence_longer_than_hint_is_reported():
     api.attn_device_status(clear=True)
     run_decode(p, max_seq_len=300)
     assert api.attn_device_status(clear=True) == 5
+
+
+def test_long_and_short_sequences_in_one_batch():
+    """A 70k-token sequence makes the workspace hold 137 splits (of 512 keys) per row; the short sequences
+    beside it take the combine's one-round-trip path (at most 16 splits, no window), the long one the
+    general path."""
+    p = inputs.paged_inputs(4, 8, 2, 128, 16, seed=78, seq_lens=[70001, 300, 1, 3000], spare_pages=4, poison=True)
+    out = run_decode(p)
+    assert api.attn_device_status(clear=True) == 0
+    ref = sdpa.decode_paged(p.q, p.k_pool, p.v_pool, p.page_table, p.seq_lens, 16, 1 / np.sqrt(128))
+    assert_parity(out, ref, "bf16", "long and short")
 
 
 def test_long_context_decode_merges_more_than_32_splits():

@@ -48,11 +48,15 @@ def test_fp8_decode_matches_oracle(case):
     assert_parity(out, ref, "bf16", str(case))
 
 
-def test_fp8_decode_equals_bf16_decode_of_the_decoded_cache():
+@pytest.mark.parametrize("Hq,Hkv,D", [(32, 8, 128), (16, 4, 64), (8, 4, 64), (16, 2, 128)],
+                         ids=["G4-D128", "G4-D64", "G2-D64", "G8-D128"])
+def test_fp8_decode_equals_bf16_decode_of_the_decoded_cache(Hq, Hkv, D):
     """With power-of-two scales every decoded element is exact in bf16 and every scaling is exact in fp32:
-    the 8-bit path must then return the bf16 path's output bit for bit, and both match the oracle."""
+    the 8-bit path must then return the bf16 path's output bit for bit, and both match the oracle.  The
+    cases cover both lane maps of the scores (two pieces per lane up to 4 heads per group, one for 8)
+    and, at D = 64, the rows whose lanes read their second piece first."""
     ks, vs = 1 / 64, 1 / 128
-    p = inputs.paged_inputs_fp8(6, 32, 8, 128, 16, seed=5, k_scale=ks, v_scale=vs,
+    p = inputs.paged_inputs_fp8(6, Hq, Hkv, D, 16, seed=5, k_scale=ks, v_scale=vs,
                                 seq_lens=[33, 1000, 17, 4097, 250, 64])
     K = torch.from_numpy(fp8.dequantize(p.k_pool, ks)).to(torch.bfloat16)
     V = torch.from_numpy(fp8.dequantize(p.v_pool, vs)).to(torch.bfloat16)
@@ -63,7 +67,7 @@ def test_fp8_decode_equals_bf16_decode_of_the_decoded_cache():
     torch.cuda.synchronize()
     assert api.attn_device_status(clear=True) == 0
     assert torch.equal(out8, out16)
-    assert_parity(out8, oracle_fp8(p, ks, vs, 1 / np.sqrt(128), 0), "bf16", "8-bit cache")
+    assert_parity(out8, oracle_fp8(p, ks, vs, 1 / np.sqrt(D), 0), "bf16", "8-bit cache")
 
 
 def test_fp8_decode_workload_every_sequence():
