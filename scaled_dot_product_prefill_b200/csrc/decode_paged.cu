@@ -51,6 +51,8 @@ constexpr float kTau = 8.0f;    // lazy-rescale threshold, log2 units
 constexpr int kStages = 2;      // ring depth per warp: 16-token K+V chunks at D = 128 (twice as many at D = 64)
 constexpr int kSplit = 1024;    // keys per split when the batch fills the GPU
 constexpr int kMinBlocks = 3;   // CTAs per SM the register allocation aims for
+// a warp's chunks of one split have their page-table entries in one lane each
+static_assert(kSplit / (kChunk * kWarps) <= 32, "at most 32 chunks per warp and split");
 
 struct DecodeParams {
   const __nv_bfloat16* q;
