@@ -278,7 +278,30 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
         }
         ++qn;
         const int kv_plane = it.b * p.Hkv + it.g;
-        auto load = [&](bool is_v, int j) -> bool {   // next ring slot <- K_j or V_j
+        // PAGED: the physical page of this lane's box of key tile j (lane rb + nb * a
+        // copies box rb of swizzle atom a), or the pool size for a box past the end
+        // of the sequence.  K_j and V_j share it, and it is read one tile ahead, so
+        // that the page-table load overlaps the wait for a free ring slot.
+        auto page_of = [&](int j) -> int {
+          if constexpr (!PAGED) {
+            return 0;
+          } else {
+            const int nb = BN / p.box_rows;
+            int ph = p.num_pages;                 // plane ph * Hkv + g is past the pool's planes
+            if (lane < nb * C::KATOMS) {
+              const int key0 = j * BN + (lane % nb) * p.box_rows;
+              if (key0 < it.skv) {
+                ph = p.page_table[static_cast<size_t>(it.b) * p.max_pages + key0 / p.page_size];
+                if (ph < 0 || ph >= p.num_pages) {  // never read outside the pool
+                  record_error(p.err, ATTN_ERRBIT_BADPAGE);
+                  ph = 0;
+                }
+              }
+            }
+            return ph;
+          }
+        };
+        auto load = [&](bool is_v, int j, int ph) -> bool {   // next ring slot <- K_j or V_j
           const int st = n % STAGES;
           if (!uni(mbar_wait(&empty[st], ((n / STAGES) & 1) ^ 1, abort_flag, p.err))) return false;
           if (lead) mbar_arrive_expect_tx(&full[st], C::TILE_BYTES);
@@ -298,14 +321,6 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
             if (lane < nb * C::KATOMS) {
               const int rb = lane % nb, a = lane / nb;
               const int key0 = j * BN + rb * p.box_rows;
-              int ph = p.num_pages;                 // plane ph * Hkv + g is past the pool's planes
-              if (key0 < it.skv) {
-                ph = p.page_table[static_cast<size_t>(it.b) * p.max_pages + key0 / p.page_size];
-                if (ph < 0 || ph >= p.num_pages) {  // never read outside the pool
-                  record_error(p.err, ATTN_ERRBIT_BADPAGE);
-                  ph = 0;
-                }
-              }
               tma_load_3d(sRing + st * C::TILE_BYTES + a * BN * 128 + rb * p.box_rows * 128, tm, &full[st],
                           a * 64, key0 % p.page_size, ph * p.Hkv + it.g);
             }
@@ -315,15 +330,23 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
         };
         // load order = the MMA thread's consumption order
         if constexpr (C::SEP_P) {   // K_lo, then K_{j+1} ahead of V_j
-          ok = load(false, it.lo_all);
+          int ph_j = page_of(it.lo_all);
+          int ph_j1 = (it.lo_all + 1 < it.hi_all) ? page_of(it.lo_all + 1) : 0;
+          ok = load(false, it.lo_all, ph_j);
           for (int j = it.lo_all; j < it.hi_all && ok; ++j) {
-            if (j + 1 < it.hi_all) ok = load(false, j + 1);
-            if (ok) ok = load(true, j);
+            const int ph_j2 = (j + 2 < it.hi_all) ? page_of(j + 2) : 0;
+            if (j + 1 < it.hi_all) ok = load(false, j + 1, ph_j1);
+            if (ok) ok = load(true, j, ph_j);
+            ph_j = ph_j1;
+            ph_j1 = ph_j2;
           }
         } else {                    // K_j, V_j
+          int ph_j = page_of(it.lo_all);
           for (int j = it.lo_all; j < it.hi_all && ok; ++j) {
-            ok = load(false, j);
-            if (ok) ok = load(true, j);
+            const int ph_j1 = (j + 1 < it.hi_all) ? page_of(j + 1) : 0;
+            ok = load(false, j, ph_j);
+            if (ok) ok = load(true, j, ph_j);
+            ph_j = ph_j1;
           }
         }
       }
