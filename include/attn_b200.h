@@ -267,7 +267,8 @@ attn_status_t attn_prefill_paged(const void* q, const void* k_pool, const void* 
  *              between calls.  Two calls in flight at once need two
  *              workspaces.
  * out        : [N, Hq, D] bf16
- * D = 128 or 64; Hq / Hkv in {1, 2, 4, 8, 16}.
+ * D = 128 or 64; Hq / Hkv in {1, 2, 4, 8} (another group size gives
+ * ATTN_ERR_UNSUPPORTED).
  *
  * Two kernels run on `stream`: a split-KV pass (one CTA per sequence, kv
  * head and span of keys; the query heads of a GQA group share every K/V

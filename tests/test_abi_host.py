@@ -97,6 +97,7 @@ def test_decode_argument_validation():
     assert decode(lib, scale=-1.0) == 1
     assert decode(lib, D=96) == 1
     assert decode(lib, Hq=24, Hkv=2) == 2               # group of 12
+    assert decode(lib, Hq=32, Hkv=2) == 2               # group of 16
     assert decode(lib, page=8) == 2
     assert decode(lib, ws=None) == 6
     need = lib.attn_decode_paged_workspace_size(4, 8, 128, 256, 16)
