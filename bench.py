@@ -51,6 +51,23 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+def tensor_peak(peaks, clocks):
+    """(peak TFLOP/s, kind) for the prefill roofline.
+
+    The burst GEMM figure is the peak of a kernel timed in a short run; when the
+    power cap held the SM clock below 97 % of its maximum during the timed steps
+    (a long run), the figure measured the same way, seconds under the cap, is
+    the comparable one.
+    """
+    burst = float(peaks["bf16_tflops"])
+    sustained = float(peaks.get("bf16_tflops_sustained", burst))
+    capped = bool("sw_power_cap" in clocks.get("reasons", []) and clocks.get("sm_mhz") and clocks.get("sm_max_mhz")
+                  and clocks["sm_mhz"] < 0.97 * clocks["sm_max_mhz"])
+    if capped:
+        return sustained, "bf16 sustained (power-capped clocks in the timed steps)"
+    return burst, "bf16 burst"
+
+
 def code_of(text):
     """C++/CUDA source with comments removed and each line's whitespace trimmed (string literals kept)."""
     import re
@@ -368,15 +385,9 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0:
         tflops = job_rate(p_flops, world, pre_ms) / 1e12
         clocks = clk.summary()
-        # The burst GEMM figure is the peak of a kernel timed in a short run; when the power cap held
-        # the SM clock down during the timed steps (a long run), the figure measured the same way,
-        # seconds under the cap, is the comparable one.  Both fractions are reported.
-        capped = ("sw_power_cap" in clocks["reasons"] and clocks["sm_mhz"] and clocks["sm_max_mhz"]
-                  and clocks["sm_mhz"] < 0.97 * clocks["sm_max_mhz"])
+        peak_t, kind_t = tensor_peak(peaks, clocks)   # both fractions are reported below
         peak_burst = float(peaks["bf16_tflops"])
         peak_sust = float(peaks.get("bf16_tflops_sustained", peak_burst))
-        peak_t = peak_sust if capped else peak_burst
-        kind_t = ("bf16 sustained (power-capped clocks in the timed steps)" if capped else "bf16 burst")
         peak_h = float(peaks["hbm_gbs"])
         ach_t = p_flops / (pre_ms * 1e-3) / 1e12
         ach_d = d_bytes / (dec_ms * 1e-3) / 1e9

@@ -93,3 +93,17 @@ def test_both_arms_describe_the_same_workload():
     lens = inputs.draw_seq_lens(d.N, d.seed, d.len_range).numpy()
     cfg = bench.arm_config(1, lens)
     assert cfg["decode"]["sum_len"] == int(lens.sum()) and cfg["workload"].startswith(bench.PREFILL.name)
+
+
+def test_tensor_peak_follows_the_clock_record():
+    """Burst peak for a short run at full clock; the sustained peak when the power cap held the clock down."""
+    peaks = {"bf16_tflops": 1650.8, "bf16_tflops_sustained": 1354.4, "hbm_gbs": 6535.7}
+    assert bench.tensor_peak(peaks, {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []})[0] == 1650.8
+    # the cap was active but did not pull the clock down: still the burst figure
+    assert bench.tensor_peak(peaks, {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]})[0] == 1650.8
+    assert bench.tensor_peak(peaks, {"sm_mhz": 1770.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]})[0] == 1354.4
+    # a clock held down with no reason (a lock) is not a power cap
+    assert bench.tensor_peak(peaks, {"sm_mhz": 1500.0, "sm_max_mhz": 1965.0, "reasons": []})[0] == 1650.8
+    assert bench.tensor_peak(peaks, {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]})[0] == 1650.8
+    assert bench.tensor_peak({"bf16_tflops": 1590.0}, {"sm_mhz": 1300.0, "sm_max_mhz": 1965.0,
+                                                        "reasons": ["sw_power_cap"]})[0] == 1590.0
